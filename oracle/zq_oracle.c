@@ -1,0 +1,319 @@
+/*
+ * zq_oracle.c -- plain, slow CPU oracle for the ZeroQuant fused quantized
+ * linear layer.  TEST INFRASTRUCTURE ONLY: only tests/, the smoke check and
+ * the bench's CPU-baseline leg may load it.  It shares no code with the CUDA
+ * library and the CUDA library never calls it.
+ *
+ * Source: "ZeroQuant: Efficient and Affordable Post-Training Quantization for
+ * Large-Scale Transformers" (arXiv 2206.01861), section-by-section summary
+ * page, Section 3.4 "Detailed, Sentence-Based Technical Breakdown":
+ *   - Eq. 2 (symmetric uniform quantizer) and its prose,
+ *   - "Group-wise Weight Quantization" (g contiguous row groups, one scale each),
+ *   - "Token-wise Activation Quantization" (one scale per token row),
+ *   - "Quantization-Optimized Transformer Kernels" (fused LN + quant, INT32
+ *     accumulator, dequantization by weight-group scale x token scale in the
+ *     GEMM epilogue, Fig. 2 fused == unfused).
+ *
+ * Readings where the pages are silent or garbled (each one is listed with its
+ * reason in the design notes of this repository):
+ *   R1 Eq. 2 as printed gives only {-1,0,1}; the prose says "normalise, then
+ *      scale to the integer range".  We use S = amax/qmax and
+ *      q = rne(x * (qmax/amax)), one IEEE fp32 division per row/group and one
+ *      fp32 multiply per element.
+ *   R2 Clamp to [-qmax, qmax] (qmax = 127 or 7): symmetric, and the absmax
+ *      scale never produces -128/-8 anyway.
+ *   R3 LayerNorm statistics are computed exactly (integer sums of x*2^24 and
+ *      of its square), so they do not depend on summation order.
+ *   R4 The fused kernel quantizes its fp16 LayerNorm output (Fig. 2: fused and
+ *      unfused compute the same output).
+ *   R5 Scales are fp32.
+ *   R6 group(o) = floor(o*g/N): g contiguous groups even when g does not
+ *      divide N.
+ *   R7 INT4: two's-complement nibbles, two per byte, low nibble = even k.
+ *   R8 "round" = round half to even.
+ *   R9 Epilogue: y = fp16( ((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]) ),
+ *      each a separate IEEE round-to-nearest op (no contraction).
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
+ * fp16 values cross the interface as their uint16 bit patterns.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#if defined(__FAST_MATH__)
+#error "the oracle must be built without fast-math"
+#endif
+
+/* ---------------------------------------------------------------- fp16 */
+
+static float h2f(uint16_t bits) {
+    _Float16 h;
+    memcpy(&h, &bits, 2);
+    return (float)h; /* exact */
+}
+
+static uint16_t f2h(float f) {
+    _Float16 h = (_Float16)f; /* IEEE round to nearest even */
+    uint16_t bits;
+    memcpy(&bits, &h, 2);
+    return bits;
+}
+
+/* Round to nearest, ties to even (R8); the default FE_TONEAREST mode. */
+static float rne(float v) { return nearbyintf(v); }
+
+static int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+/* ------------------------------------------- Eq. 2, one scale per set */
+
+/* The symmetric quantizer of Eq. 2 under readings R1, R2, R8 for one set of
+ * values that shares one scale (a weight group or a token row).
+ * amax is max|x| over the set; returns S and writes inv = qmax/amax. */
+static float eq2_scale(float amax, int qmax, float *inv) {
+    if (amax == 0.0f) {
+        *inv = 0.0f;
+        return 0.0f;
+    }
+    *inv = (float)qmax / amax;
+    return amax / (float)qmax;
+}
+
+static int eq2_quantize(float x, float inv, int qmax) {
+    if (inv == 0.0f) return 0;
+    float v = x * inv;
+    return clampi((int)rne(v), -qmax, qmax);
+}
+
+/* ------------------------------------- group-wise weight quantization */
+
+/* Group index of output row o when N rows are split into g contiguous
+ * groups (R6). */
+int zqo_group_of(int o, int N, int g) { return (int)(((int64_t)o * g) / N); }
+
+/* W: fp16 bits [N*K] row-major, rows = outputs.  bits = 8 or 4.
+ * q: int8 [N*K] (values in [-qmax, qmax]); s_grp: fp32 [g].
+ * Returns 0, or -1 on bad arguments. */
+int zqo_quantize_weights_groupwise(const uint16_t *W, int N, int K, int g, int bits,
+                                   int8_t *q, float *s_grp) {
+    if (N < 1 || K < 1 || g < 1 || g > N || (bits != 8 && bits != 4)) return -1;
+    const int qmax = bits == 8 ? 127 : 7;
+    float *amax = (float *)calloc((size_t)g, sizeof(float));
+    if (!amax) return -1;
+    /* S_i = max|W_i| over the rows of group i */
+    for (int o = 0; o < N; ++o) {
+        int gi = zqo_group_of(o, N, g);
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(h2f(W[(size_t)o * K + k]));
+            if (a > amax[gi]) amax[gi] = a;
+        }
+    }
+    float *inv = (float *)malloc((size_t)g * sizeof(float));
+    if (!inv) { free(amax); return -1; }
+    for (int i = 0; i < g; ++i) s_grp[i] = eq2_scale(amax[i], qmax, &inv[i]);
+    for (int o = 0; o < N; ++o) {
+        int gi = zqo_group_of(o, N, g);
+        for (int k = 0; k < K; ++k)
+            q[(size_t)o * K + k] = (int8_t)eq2_quantize(h2f(W[(size_t)o * K + k]), inv[gi], qmax);
+    }
+    free(inv);
+    free(amax);
+    return 0;
+}
+
+/* R7: byte j of row o = (q[o,2j] & 0xF) | ((q[o,2j+1] & 0xF) << 4).  K even. */
+int zqo_pack_int4(const int8_t *q, int N, int K, uint8_t *packed) {
+    if (K % 2) return -1;
+    for (int o = 0; o < N; ++o)
+        for (int j = 0; j < K / 2; ++j) {
+            unsigned lo = (unsigned)q[(size_t)o * K + 2 * j] & 0xFu;
+            unsigned hi = (unsigned)q[(size_t)o * K + 2 * j + 1] & 0xFu;
+            packed[(size_t)o * (K / 2) + j] = (uint8_t)(lo | (hi << 4));
+        }
+    return 0;
+}
+
+/* Inverse of zqo_pack_int4: sign-extend each nibble. */
+int zqo_unpack_int4(const uint8_t *packed, int N, int K, int8_t *q) {
+    if (K % 2) return -1;
+    for (int o = 0; o < N; ++o)
+        for (int j = 0; j < K / 2; ++j) {
+            unsigned b = packed[(size_t)o * (K / 2) + j];
+            int lo = (int)(b & 0xFu), hi = (int)(b >> 4);
+            q[(size_t)o * K + 2 * j] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+            q[(size_t)o * K + 2 * j + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+        }
+    return 0;
+}
+
+/* -------------------------------------------- LayerNorm (reading R3) */
+
+/* Exact row statistics: a_k = x_k * 2^24 is an integer (|a_k| < 2^40) for
+ * every finite fp16 x_k.  S1 = sum a_k (int64), S2 = sum a_k^2 (128-bit,
+ * returned as two 64-bit halves). */
+void zqo_ln_exact_sums(const uint16_t *x, int K, int64_t *S1, uint64_t *S2_hi, uint64_t *S2_lo) {
+    int64_t s1 = 0;
+    unsigned __int128 s2 = 0;
+    for (int k = 0; k < K; ++k) {
+        int64_t a = (int64_t)((double)h2f(x[k]) * 16777216.0); /* exact */
+        s1 += a;
+        unsigned __int128 m = (unsigned __int128)(a < 0 ? -a : a);
+        s2 += m * m;
+    }
+    *S1 = s1;
+    *S2_hi = (uint64_t)(s2 >> 64);
+    *S2_lo = (uint64_t)s2;
+}
+
+/* mean and rstd of one row, from the exact sums (biased variance, /K). */
+void zqo_ln_row_stats(const uint16_t *x, int K, float eps, float *mean_out, float *rstd_out,
+                      double *mean_d_out, double *var_d_out) {
+    int64_t S1;
+    uint64_t hi, lo;
+    zqo_ln_exact_sums(x, K, &S1, &hi, &lo);
+    double mean_d = ((double)S1 * 0x1p-24) / (double)K;
+    double e2_d = (((double)hi * 0x1p64 + (double)lo) * 0x1p-48) / (double)K;
+    double msq = mean_d * mean_d;
+    double var_d = e2_d - msq;
+    if (var_d < 0.0) var_d = 0.0;
+    double denom = sqrt(var_d + (double)eps);
+    *rstd_out = (float)(1.0 / denom);
+    *mean_out = (float)mean_d;
+    if (mean_d_out) *mean_d_out = mean_d;
+    if (var_d_out) *var_d_out = var_d;
+}
+
+/* Unfused step 1 of Fig. 2: y = fp16(LN(x)) per row.  gamma/beta may be
+ * NULL (gamma = NULL means the identity: y = x, the quant-only mode). */
+int zqo_layernorm(const uint16_t *X, const uint16_t *gamma, const uint16_t *beta, int T, int K,
+                  float eps, uint16_t *Y) {
+    if (T < 0 || K < 1) return -1;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *x = X + (size_t)t * K;
+        uint16_t *y = Y + (size_t)t * K;
+        if (!gamma) {
+            memcpy(y, x, (size_t)K * 2);
+            continue;
+        }
+        float mean, rstd;
+        zqo_ln_row_stats(x, K, eps, &mean, &rstd, NULL, NULL);
+        for (int k = 0; k < K; ++k) {
+            float d = h2f(x[k]) - mean;
+            float n = d * rstd;
+            float s = n * h2f(gamma[k]);
+            float b = beta ? h2f(beta[k]) : 0.0f;
+            y[k] = f2h(s + b);
+        }
+    }
+    return 0;
+}
+
+/* Unfused step 2 of Fig. 2: token-wise symmetric INT8 quantization of fp16
+ * rows, one scale per row (Token-wise Activation Quantization). */
+int zqo_token_quant(const uint16_t *Y, int T, int K, int8_t *q, float *s_tok) {
+    if (T < 0 || K < 1) return -1;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *y = Y + (size_t)t * K;
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float a = fabsf(h2f(y[k]));
+            if (a > amax) amax = a;
+        }
+        float inv;
+        s_tok[t] = eq2_scale(amax, 127, &inv);
+        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(y[k]), inv, 127);
+    }
+    return 0;
+}
+
+/* The fused LN + token quantization of Fig. 2 (right), written as its own
+ * single pass per row so that the Fig. 2 equality (fused == unfused) is a
+ * real check.  Y_ln may be NULL. */
+int zqo_ln_quant(const uint16_t *X, const uint16_t *gamma, const uint16_t *beta, int T, int K,
+                 float eps, int8_t *q, float *s_tok, uint16_t *Y_ln) {
+    if (T < 0 || K < 1) return -1;
+    uint16_t *row = (uint16_t *)malloc((size_t)K * 2);
+    if (!row) return -1;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *x = X + (size_t)t * K;
+        float mean = 0.0f, rstd = 1.0f;
+        if (gamma) zqo_ln_row_stats(x, K, eps, &mean, &rstd, NULL, NULL);
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            uint16_t yb;
+            if (gamma) {
+                float v = ((h2f(x[k]) - mean) * rstd) * h2f(gamma[k]);
+                yb = f2h(v + (beta ? h2f(beta[k]) : 0.0f));
+            } else {
+                yb = x[k];
+            }
+            row[k] = yb;
+            float a = fabsf(h2f(yb));
+            if (a > amax) amax = a;
+        }
+        float inv;
+        s_tok[t] = eq2_scale(amax, 127, &inv);
+        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(row[k]), inv, 127);
+        if (Y_ln) memcpy(Y_ln + (size_t)t * K, row, (size_t)K * 2);
+    }
+    free(row);
+    return 0;
+}
+
+/* ------------------------------------------------ INT32 GEMM (exact) */
+
+/* acc[t,o] = sum_k xq[t,k]*wq[o,k], summed in int64 and checked to fit
+ * int32 (the INT32 accumulator of the INT8 GEMM).  Returns 0, or -2 if a
+ * sum does not fit int32. */
+int zqo_gemm_i32(const int8_t *xq, const int8_t *wq, int T, int N, int K, int32_t *acc) {
+    for (int t = 0; t < T; ++t)
+        for (int o = 0; o < N; ++o) {
+            int64_t s = 0;
+            const int8_t *a = xq + (size_t)t * K, *b = wq + (size_t)o * K;
+            for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];
+            if (s > INT32_MAX || s < INT32_MIN) return -2;
+            acc[(size_t)t * N + o] = (int32_t)s;
+        }
+    return 0;
+}
+
+/* ----------------------------------------------- dequant epilogue (R9) */
+
+/* y[t,o] = fp16( ((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]) ).
+ * bias may be NULL (treated as 0). */
+int zqo_dequant(const int32_t *acc, const float *s_tok, const float *s_grp, int g,
+                const uint16_t *bias, int T, int N, uint16_t *Y) {
+    if (g < 1 || g > N) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int o = 0; o < N; ++o) {
+            float a = (float)acc[(size_t)t * N + o];
+            float v = a * s_tok[t];
+            v = v * s_grp[zqo_group_of(o, N, g)];
+            v = v + (bias ? h2f(bias[o]) : 0.0f);
+            Y[(size_t)t * N + o] = f2h(v);
+        }
+    return 0;
+}
+
+/* GEMM + dequant for one token row at a time (the fused form of Fig. 2,
+ * written without an int32 intermediate buffer). */
+int zqo_linear_q(const int8_t *xq, const float *s_tok, const int8_t *wq, const float *s_grp, int g,
+                 const uint16_t *bias, int T, int N, int K, uint16_t *Y) {
+    if (g < 1 || g > N) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int o = 0; o < N; ++o) {
+            int64_t s = 0;
+            for (int k = 0; k < K; ++k) s += (int64_t)xq[(size_t)t * K + k] * wq[(size_t)o * K + k];
+            if (s > INT32_MAX || s < INT32_MIN) return -2;
+            float v = (float)(int32_t)s * s_tok[t];
+            v = v * s_grp[zqo_group_of(o, N, g)];
+            v = v + (bias ? h2f(bias[o]) : 0.0f);
+            Y[(size_t)t * N + o] = f2h(v);
+        }
+    return 0;
+}
+
+/* Reports the rounding mode so a test can confirm round-to-nearest. */
+int zqo_rounding_is_nearest(void) { return fegetround() == FE_TONEAREST; }

@@ -1,0 +1,59 @@
+"""The pins must reject a plausibly wrong oracle.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU),
+builds it, and runs the pin suite against that build; the suite must fail.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle.zq_oracle as zo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "round_down": ("return nearbyintf(v);", "return floorf(v);"),
+    "ties_away": ("return nearbyintf(v);", "return roundf(v);"),
+    "scale_qmax_plus_one": ("return amax / (float)qmax;", "return amax / (float)(qmax + 1);"),
+    "group_ceil": ("return (int)(((int64_t)o * g) / N);", "return (int)(((int64_t)o * g + N - 1) / N);"),
+    "nibble_shift": ("(uint8_t)(lo | (hi << 4))", "(uint8_t)((lo << 4) | hi)"),
+    "ln_mean_sign": ("float d = h2f(x[k]) - mean;", "float d = h2f(x[k]) + mean;"),
+    "ln_var_drop_mean": ("double var_d = e2_d - msq;", "double var_d = e2_d;"),
+    "ln_unbiased_var": ("double e2_d = (((double)hi * 0x1p64 + (double)lo) * 0x1p-48) / (double)K;",
+                        "double e2_d = (((double)hi * 0x1p64 + (double)lo) * 0x1p-48) / (double)(K - 1);"),
+    "gemm_reversed_k": ("for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];",
+                        "for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[K - 1 - k];"),
+    "dequant_row_scale_swapped": ("v = v * s_grp[zqo_group_of(o, N, g)];\n            v = v + (bias ? h2f(bias[o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM + dequant",
+                                  "v = v * s_grp[zqo_group_of(N - 1 - o, N, g)];\n            v = v + (bias ? h2f(bias[o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM + dequant"),
+    "dequant_bias_reversed": ("v = v + (bias ? h2f(bias[o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM",
+                              "v = v + (bias ? h2f(bias[N - 1 - o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM"),
+    "token_clamp_126": ("s_tok[t] = eq2_scale(amax, 127, &inv);\n        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(y[k]), inv, 127);",
+                        "s_tok[t] = eq2_scale(amax, 127, &inv);\n        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(y[k]), inv, 126);"),
+}
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    src = open(zo._SRC).read()
+    d = tmp_path_factory.mktemp("mutants")
+    procs = {}
+    for name, (old, new) in MUTATIONS.items():
+        assert src.count(old) == 1, name
+        c = d / f"{name}.c"
+        c.write_text(src.replace(old, new))
+        so = d / f"{name}.so"
+        subprocess.check_call(["gcc", *zo.CFLAGS, str(c), "-o", str(so), "-lm"])
+        env = dict(os.environ, ZQ_ORACLE_LIB=str(so))
+        procs[name] = subprocess.Popen(
+            [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+             os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+            cwd=ROOT, env=env, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
+    return {name: (p.wait(timeout=600), p.stdout.read().decode()) for name, p in procs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_reject_mutant(mutant_runs, name):
+    rc, out = mutant_runs[name]
+    assert rc == 1, f"mutant {name} was not caught (rc={rc}):\n{out[-2000:]}"

@@ -1,0 +1,366 @@
+"""Pins of the CPU oracle against what the paper and the mathematics fix.
+
+Each test checks the oracle against something other than itself: an error
+bound that Eq. 2 implies, an exact round trip, a brute-force integer sum, a
+library routine (numpy int64 matmul, torch fp64 layer_norm), exact rational
+arithmetic, or a figure printed in the paper (tests/golden/).  Citations are
+to "ZeroQuant" (arXiv 2206.01861), section-by-section summary, Sec. 3.4.
+"""
+from fractions import Fraction
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int4_quantized_transformer_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+def _ulp16(v):
+    """Spacing of fp16 numbers at |v| (for normal and subnormal values)."""
+    v = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(v, 2.0 ** -14)))
+    return 2.0 ** (e - 10)
+
+
+def _eq2_bound(S, qmax):
+    # |x - q*S| <= S*(1/2 + 3*qmax*2^-24): the rounding of q plus the three
+    # fp32 roundings (qmax/amax, amax/qmax, x*inv) of the symmetric quantizer.
+    return np.asarray(S, np.float64) * (0.5 + 3.0 * qmax * 2.0 ** -24)
+
+
+# --------------------------------------------------------------------- weights
+
+@pytest.mark.parametrize("N,K,g,bits", [(256, 64, 4, 8), (1024, 96, 48, 8), (96, 64, 7, 4),
+                                        (64, 32, 64, 4), (50, 16, 1, 8)])
+def test_weight_quant_error_bound_and_saturation(N, K, g, bits):
+    """Eq. 2 with S_i = max|W_i|/qmax: every element within S_i/2, and the
+    largest element of each non-zero group maps to +-qmax (Sec. 3.4,
+    "Group-wise Weight Quantization")."""
+    qmax = 127 if bits == 8 else 7
+    row_scale = np.exp(RNG.normal(0, 1.0, size=(N, 1)))  # rows with ~10x range spread
+    W = (RNG.normal(0, 0.02, size=(N, K)) * row_scale).astype(np.float16)
+    q, s = oracle.quantize_weights_groupwise(W, g, bits)
+    assert q.shape == (N, K) and s.shape == (g,)
+    grp = oracle.group_index(N, g)
+    S = s[grp][:, None].astype(np.float64)
+    err = np.abs(W.astype(np.float64) - q.astype(np.float64) * S)
+    assert np.all(err <= _eq2_bound(S, qmax))
+    assert np.all(np.abs(q) <= qmax)
+    for i in range(g):
+        rows = q[grp == i]
+        assert np.abs(rows).max() == qmax
+        # the scale is the group's own absmax / qmax, up to one fp32 rounding
+        amax = np.abs(W[grp == i].astype(np.float64)).max()
+        assert abs(s[i] - amax / qmax) <= 2.0 ** -23 * amax / qmax
+
+
+def test_group_partition_properties():
+    """g contiguous groups of floor(N/g) or ceil(N/g) rows, in order, and
+    N/g rows each when g divides N (Sec. 3.4: g groups of n/g rows)."""
+    for N, g in [(256, 4), (1024, 48), (768, 48), (6144, 192), (7, 7), (9, 1), (1000, 3)]:
+        grp = oracle.group_index(N, g)
+        assert grp[0] == 0 and grp[-1] == g - 1
+        assert np.all(np.diff(grp) >= 0) and np.all(np.diff(grp) <= 1)
+        sizes = np.bincount(grp, minlength=g)
+        assert sizes.min() >= N // g and sizes.max() <= -(-N // g) and sizes.sum() == N
+        if N % g == 0:
+            assert np.all(sizes == N // g)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_weight_quant_on_grid_round_trip(bits):
+    """Weights already on the grid k*S come back exactly: S = 2^-7 (INT8) or
+    2^-3 (INT4) when each group holds its +-qmax*S extreme."""
+    qmax, S = (127, 2.0 ** -7) if bits == 8 else (7, 2.0 ** -3)
+    N, K, g = 48, 32, 6
+    k = RNG.integers(-qmax, qmax + 1, size=(N, K))
+    grp = oracle.group_index(N, g)
+    for i in range(g):
+        r = np.nonzero(grp == i)[0][0]
+        k[r, 0] = qmax if i % 2 else -qmax
+    W = (k * S).astype(np.float16)
+    q, s = oracle.quantize_weights_groupwise(W, g, bits)
+    assert np.array_equal(q, k.astype(np.int8))
+    assert np.all(s == np.float32(S))
+
+
+def test_weight_quant_zero_group_and_tiny_case():
+    """A zero group has scale 0 and codes 0; a 4x4 case checked by hand."""
+    W = np.array([[0.5, -0.25, 0.125, 0.0],
+                  [0.0, 0.0, 0.0, -1.0],
+                  [0.0, 0.0, 0.0, 0.0],
+                  [0.0, 0.0, 0.0, 0.0]], np.float16)
+    q, s = oracle.quantize_weights_groupwise(W, 2, 8)
+    # group 0 = rows 0,1, amax 1.0 -> S = 1/127, q = rne(w*127)
+    assert s[0] == np.float32(1.0) / np.float32(127.0)
+    assert q[0].tolist() == [64, -32, 16, 0]  # 63.5 -> 64 (tie to even), 31.75 -> 32, 15.875 -> 16
+    assert q[1].tolist() == [0, 0, 0, -127]
+    assert s[1] == 0.0 and not q[2:].any()
+    q4, s4 = oracle.quantize_weights_groupwise(W, 2, 4)
+    # INT4: q = rne(w*7): 3.5 -> 4 (tie to even), -1.75 -> -2, 0.875 -> 1
+    assert q4[0].tolist() == [4, -2, 1, 0] and q4[1].tolist() == [0, 0, 0, -7]
+
+
+def test_round_half_to_even_ties():
+    """Ties go to even (reading R8): x*inv = 0.5, 1.5, 2.5 -> 0, 2, 2."""
+    W = np.array([[127.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5]], np.float16)
+    q, s = oracle.quantize_weights_groupwise(W, 1, 8)
+    assert s[0] == np.float32(1.0)
+    assert q[0].tolist() == [127, 0, 2, 2, 0, -2, -2, 126]
+    assert oracle.rounding_is_nearest()
+
+
+# ------------------------------------------------------------------------ int4
+
+def test_int4_pack_golden_and_round_trip():
+    rows = []
+    with open(os.path.join(GOLDEN, "int4_pack.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                a, b, byte = line.split()
+                rows.append((int(a), int(b), int(byte, 16)))
+    q = np.array([[a, b] for a, b, _ in rows], np.int8).reshape(1, -1)
+    packed = oracle.pack_int4(q)
+    assert packed.tolist()[0] == [byte for _, _, byte in rows]
+    # every nibble pair survives pack -> unpack
+    vals = np.arange(-8, 8)
+    pairs = np.array(np.meshgrid(vals, vals)).reshape(2, -1).T.reshape(1, -1).astype(np.int8)
+    p = oracle.pack_int4(pairs)
+    assert p.nbytes == pairs.size // 2
+    assert np.array_equal(oracle.unpack_int4(p, pairs.shape[1]), pairs)
+
+
+# ------------------------------------------------------------------- LayerNorm
+
+def test_ln_exact_sums_brute_force():
+    """S1, S2 equal Python big-int sums of x*2^24 (tiny rows, incl. extremes)."""
+    for row in [np.array([1.0, -2.0, 0.5, 65504.0, -65504.0, 2.0 ** -24], np.float16),
+                RNG.normal(0, 3, 37).astype(np.float16), np.zeros(5, np.float16)]:
+        s1, s2 = oracle.ln_exact_sums(row)
+        a = [int(Fraction(float(v)) * 2 ** 24) for v in row]
+        assert s1 == sum(a) and s2 == sum(v * v for v in a)
+
+
+def test_ln_stats_against_exact_rationals():
+    """mean and biased variance equal the exact rational values to ~1 ulp."""
+    for K in (7, 64, 768, 4096):
+        x = synth.activations(1, K, seed=K, n_outliers=3, outlier_scale=20.0).numpy()[0]
+        mean_f, rstd_f, mean_d, var_d = oracle.ln_row_stats(x, 1e-5)
+        xs = [Fraction(float(v)) for v in x]
+        m = sum(xs) / K
+        var = sum(v * v for v in xs) / K - m * m
+        assert abs(mean_d - float(m)) <= 4 * 2.0 ** -52 * (abs(float(m)) + 2.0 ** -40)
+        assert abs(var_d - float(var)) <= 1e-12 * float(var)
+        assert abs(float(rstd_f) - 1.0 / np.sqrt(float(var) + 1e-5)) <= 2.0 ** -23 * float(rstd_f)
+
+
+def test_layernorm_against_torch_fp64():
+    """fp16(LN(x)) agrees with torch.nn.functional.layer_norm computed in
+    float64 and rounded once: never more than 1 fp16 ulp apart, equal almost
+    everywhere (the oracle rounds in fp32 between steps)."""
+    T, K = 33, 768
+    X = synth.activations(T, K, seed=5, n_outliers=6, outlier_scale=20.0)
+    gamma, beta = synth.ln_params(K, 6)
+    y = oracle.layernorm(X.numpy(), gamma.numpy(), beta.numpy(), 1e-5).astype(np.float64)
+    ref = torch.nn.functional.layer_norm(X.double(), (K,), gamma.double(), beta.double(), 1e-5)
+    ref16 = ref.to(torch.float16).double().numpy()
+    diff = np.abs(y - ref16)
+    assert np.all(diff <= _ulp16(ref16) * 1.0001)
+    assert (diff == 0).mean() > 0.99
+
+
+def test_layernorm_constant_row_gives_beta():
+    K = 64
+    x = np.full((2, K), 3.25, np.float16)
+    gamma, beta = synth.ln_params(K, 9)
+    y = oracle.layernorm(x, gamma.numpy(), beta.numpy(), 1e-5)
+    assert np.array_equal(y[0], beta.numpy()) and np.array_equal(y[1], beta.numpy())
+
+
+# -------------------------------------------------------------- token quant
+
+def test_token_quant_bound_saturation_and_zero_rows():
+    """Sec. 3.4 "Token-wise Activation Quantization": one scale per token row,
+    S = max|x_token|/127, every element within S/2, extremes at +-127, zero
+    rows give S = 0 and all-zero codes."""
+    T, K = 40, 256
+    Y = synth.activations(T, K, seed=3, n_outliers=6, outlier_scale=20.0).numpy()
+    Y[5] = 0
+    q, s = oracle.token_quant(Y)
+    assert s.shape == (T,)
+    S = s[:, None].astype(np.float64)
+    assert np.all(np.abs(Y.astype(np.float64) - q * S) <= _eq2_bound(S, 127))
+    for t in range(T):
+        if t == 5:
+            assert s[t] == 0 and not q[t].any()
+        else:
+            assert np.abs(q[t]).max() == 127
+            amax = np.abs(Y[t].astype(np.float64)).max()
+            assert abs(s[t] - amax / 127) <= 2.0 ** -23 * amax / 127
+
+
+def test_token_quant_on_grid_round_trip():
+    T, K = 8, 64
+    k = RNG.integers(-127, 128, size=(T, K))
+    k[:, 3] = 127
+    Y = (k * 2.0 ** -7).astype(np.float16)
+    q, s = oracle.token_quant(Y)
+    assert np.array_equal(q, k.astype(np.int8)) and np.all(s == np.float32(2.0 ** -7))
+
+
+@pytest.mark.parametrize("kind", ["normal", "zero_rows", "constant_rows", "max_values", "tiny_values"])
+@pytest.mark.parametrize("with_ln", [True, False])
+def test_fused_equals_unfused_fig2(kind, with_ln):
+    """Fig. 2: LN+Quant fused produces the same output as LN then Quant."""
+    T, K = 24, 192
+    X = synth.edge_activations(kind, T, K).numpy()
+    gamma, beta = synth.ln_params(K, 11) if with_ln else (None, None)
+    g = None if gamma is None else gamma.numpy()
+    b = None if beta is None else beta.numpy()
+    q, s, y = oracle.ln_quant(X, g, b, 1e-5, want_y=True)
+    y2 = oracle.layernorm(X, g, b, 1e-5)
+    q2, s2 = oracle.token_quant(y2)
+    assert np.array_equal(y.view(np.uint16), y2.view(np.uint16))
+    assert np.array_equal(q, q2) and np.array_equal(s.view(np.uint32), s2.view(np.uint32))
+
+
+# ------------------------------------------------------------------- GEMM
+
+def test_gemm_brute_force_tiny():
+    for T, N, K in [(1, 1, 1), (3, 5, 7), (8, 8, 8), (2, 3, 64)]:
+        a = RNG.integers(-127, 128, size=(T, K)).astype(np.int8)
+        b = RNG.integers(-127, 128, size=(N, K)).astype(np.int8)
+        acc = oracle.gemm_i32(a, b)
+        for t in range(T):
+            for o in range(N):
+                assert acc[t, o] == sum(int(a[t, k]) * int(b[o, k]) for k in range(K))
+
+
+def test_gemm_matches_numpy_int64():
+    a = RNG.integers(-127, 128, size=(16, 64)).astype(np.int8)
+    b = RNG.integers(-7, 8, size=(256, 64)).astype(np.int8)
+    acc = oracle.gemm_i32(a, b)
+    assert np.array_equal(acc, a.astype(np.int64) @ b.astype(np.int64).T)
+    assert np.abs(acc).max() <= 127 * 7 * 64
+
+
+def test_gemm_int32_overflow_limit():
+    """127*127*K fits int32 up to K = 133144 and not beyond."""
+    for K, ok in [(133144, True), (133145, False)]:
+        a = np.full((1, K), 127, np.int8)
+        if ok:
+            assert oracle.gemm_i32(a, a)[0, 0] == 127 * 127 * K
+        else:
+            with pytest.raises(OverflowError):
+                oracle.gemm_i32(a, a)
+
+
+# -------------------------------------------------------------- epilogue
+
+def test_dequant_special_cases():
+    T, N, g = 3, 8, 2
+    bias = synth.bias(N, 4).numpy()
+    s_tok = np.array([0.5, 0.25, 2.0], np.float32)
+    s_grp = np.array([0.125, 4.0], np.float32)
+    y = oracle.dequant(np.zeros((T, N), np.int32), s_tok, s_grp, bias)
+    assert np.array_equal(y, np.broadcast_to(bias, (T, N)))  # acc = 0 -> bias
+    acc = np.arange(T * N, dtype=np.int32).reshape(T, N) - 7
+    y = oracle.dequant(acc, np.ones(T, np.float32), np.ones(g, np.float32), None)
+    assert np.array_equal(y, acc.astype(np.float16))  # unit scales -> fp16(acc)
+    y = oracle.dequant(np.array([[2049, 2051, -2049]], np.int32), np.ones(1, np.float32),
+                       np.ones(1, np.float32), None)
+    assert y.tolist() == [[2048.0, 2052.0, -2048.0]]  # fp16 ties to even
+
+
+def test_dequant_against_fp64_closed_form():
+    """y[t,o] = acc*s_tok[t]*s_grp[group(o)] + b[o], within one fp16 rounding
+    plus fp32 rounding: distinct per-row and per-group scales catch a swapped
+    or transposed scale."""
+    T, N, g = 9, 96, 7
+    acc = RNG.integers(-2 ** 20, 2 ** 20, size=(T, N)).astype(np.int32)
+    s_tok = RNG.uniform(1e-3, 1e-1, T).astype(np.float32)
+    s_grp = RNG.uniform(1e-4, 1e-2, g).astype(np.float32)
+    bias = synth.bias(N, 8).numpy()
+    y = oracle.dequant(acc, s_tok, s_grp, bias).astype(np.float64)
+    grp = oracle.group_index(N, g)
+    ref = acc * s_tok[:, None].astype(np.float64) * s_grp[grp][None, :] + bias.astype(np.float64)
+    assert np.all(np.abs(y - ref) <= 0.5 * _ulp16(ref) + 8 * 2.0 ** -24 * np.abs(ref) + 1e-7)
+
+
+def test_linear_q_equals_gemm_then_dequant():
+    """Fig. 2: GEMM+Dequant fused == GEMM then Dequant."""
+    a = RNG.integers(-127, 128, size=(13, 160)).astype(np.int8)
+    b = RNG.integers(-127, 128, size=(72, 160)).astype(np.int8)
+    s_tok = RNG.uniform(1e-3, 1e-1, 13).astype(np.float32)
+    s_grp = RNG.uniform(1e-4, 1e-2, 5).astype(np.float32)
+    bias = synth.bias(72, 1).numpy()
+    y1 = oracle.linear_q(a, s_tok, b, s_grp, bias)
+    y2 = oracle.dequant(oracle.gemm_i32(a, b), s_tok, s_grp, bias)
+    assert np.array_equal(y1.view(np.uint16), y2.view(np.uint16))
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_quantized_linear_within_quantization_error(bits):
+    """End to end: the quantized layer approximates X W^T + b (fp64) within
+    the error that Eq. 2 allows on each operand, element by element."""
+    layer = "tiny"
+    gi = synth.gemm_inputs(layer, 0, 16)
+    X, W, b = gi.X.numpy(), gi.W.numpy(), gi.b.numpy()
+    xq, s_tok = oracle.ln_quant(X)
+    wq, s_grp = oracle.quantize_weights_groupwise(W, gi.spec.g, bits)
+    y = oracle.linear_q(xq, s_tok, wq, s_grp, b).astype(np.float64)
+    Xd, Wd = X.astype(np.float64), W.astype(np.float64)
+    ref = Xd @ Wd.T + b.astype(np.float64)
+    qmax = 127 if bits == 8 else 7
+    dx = _eq2_bound(s_tok, 127)[:, None]  # per token
+    dw = _eq2_bound(s_grp[oracle.group_index(W.shape[0], gi.spec.g)], qmax)[:, None]  # per out row
+    bound = (np.abs(Xd).sum(1, keepdims=True) * dw.T + dx * np.abs(Wd).sum(1)[None, :]
+             + dx * dw.T * X.shape[1])
+    bound = bound * (1 + 1e-5) + _ulp16(ref) + 1e-6
+    assert np.all(np.abs(y - ref) <= bound)
+
+
+# ------------------------------------------------------------------ bytes
+
+def _golden_bytes():
+    d = {}
+    with open(os.path.join(GOLDEN, "paper_bytes.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                k, v = line.split()
+                d[k] = float(v)
+    return d
+
+
+def test_scale_memory_example():
+    """Sec. 3.4: 4096x4096 in 64 groups -> 64 FP16 scales = 128 B vs 32 MB."""
+    d = _golden_bytes()
+    N, K, g = int(d["scale_example_rows"]), int(d["scale_example_cols"]), int(d["scale_example_groups"])
+    W = np.zeros((N, K), np.float16)
+    W[:, 0] = 1.0
+    q, s = oracle.quantize_weights_groupwise(W, g, 8)
+    assert s.size == g
+    assert s.size * 2 == d["scale_example_fp16_scale_bytes"]  # the paper's fp16 scales
+    assert s.nbytes == 2 * d["scale_example_fp16_scale_bytes"]  # this library keeps fp32 scales
+    assert W.nbytes == d["scale_example_fp16_weight_bytes"]
+
+
+def test_w48_footprint_is_about_three_times_smaller():
+    """Sec. 1 / 6.3: INT4 FFN + INT8 attention ~ 3x smaller than FP16."""
+    d = _golden_bytes()
+    L = synth.LAYERS["gpt350m"]
+    q_bytes = fp16_bytes = 0
+    for s in L.gemms:
+        W = np.zeros((s.N, s.K), np.float16)
+        q, sc = oracle.quantize_weights_groupwise(W, s.g, s.bits)
+        packed = oracle.pack_int4(q) if s.bits == 4 else q
+        q_bytes += packed.nbytes + sc.nbytes
+        fp16_bytes += W.nbytes
+    assert abs(fp16_bytes / q_bytes - d["w48_vs_fp16_ratio"]) < 0.01 * d["w48_vs_fp16_ratio"]

@@ -1,0 +1,161 @@
+/*
+ * zq.h -- C ABI of libzq, the B200 (sm_100a) fused quantized linear layer of
+ * ZeroQuant ("ZeroQuant: Efficient and Affordable Post-Training Quantization
+ * for Large-Scale Transformers", arXiv 2206.01861).
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - All tensor pointers are DEVICE pointers into memory the caller owns and
+ *    keeps alive until the work queued on `stream` has finished.  fp16 tensors
+ *    are passed as `void*` holding IEEE binary16 values.
+ *  - Matrices are row-major and dense: X[T][K] (tokens x hidden),
+ *    W[N][K] (output features x hidden; the paper's W in R^{n x m} with one
+ *    row per output), Y[T][N].
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and on the device that is current for the calling thread.
+ *  - Argument errors are reported synchronously (ZQ_ERR_NULL / _SHAPE /
+ *    _ALIGN / _UNSUPPORTED) and nothing is launched.  Launch failures return
+ *    ZQ_ERR_CUDA.  A kernel that gives up a bounded device-side wait records
+ *    the fact in a per-device status word that zq_device_status() reports.
+ *  - Group of output row o when N rows are split into g contiguous groups:
+ *    group(o) = floor(o*g/N).
+ *  - Rounding: round half to even everywhere; every floating-point step is a
+ *    single IEEE round-to-nearest operation (no fused multiply-add), so the
+ *    results are bit-for-bit reproducible.
+ */
+#ifndef ZQ_H_
+#define ZQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t */
+typedef struct CUstream_st* zq_stream_t;
+
+typedef enum {
+  ZQ_OK = 0,
+  ZQ_ERR_NULL = 1,        /* a required pointer is NULL */
+  ZQ_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  ZQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  ZQ_ERR_UNSUPPORTED = 4, /* valid request this build does not handle (e.g. bits) */
+  ZQ_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
+  ZQ_ERR_TIMEOUT = 6      /* a kernel gave up a bounded wait (zq_device_status) */
+} zq_status;
+
+/* Human-readable name of a status code (static storage). */
+const char* zq_status_str(int status);
+
+/* ABI version of this header (major*100 + minor). */
+int zq_abi_version(void);
+
+/*
+ * zq_quantize_weights_groupwise -- offline group-wise symmetric weight
+ * quantization (Sec. 3.4 "Group-wise Weight Quantization", Eq. 2).
+ *   W      fp16 [N][K]; N rows split into g contiguous groups.
+ *   bits   8: Wq is int8 [N][K].  4: Wq is uint8 [N][K/2], two signed
+ *          two's-complement nibbles per byte, low nibble = even k.
+ *   s_grp  fp32 [g]: S_i = amax_i / qmax with amax_i = max |W| over group i,
+ *          qmax = 127 (bits 8) or 7 (bits 4).  q = clamp(rne(w * (qmax/amax_i)),
+ *          -qmax, qmax); a group that is all zero gets S_i = 0 and q = 0.
+ * Requirements: 1 <= g <= N, K >= 1, K % 16 == 0 (K % 32 == 0 for bits 4),
+ * pointers 16-byte aligned.
+ */
+zq_status zq_quantize_weights_groupwise(const void* W, int N, int K, int g, int bits, void* Wq,
+                                        float* s_grp, zq_stream_t stream);
+
+/*
+ * zq_ln_quant -- fused LayerNorm + token-wise dynamic INT8 quantization
+ * (Sec. 3.4 "Token-wise Activation Quantization" and "Kernel fusion for
+ * token-wise activation quantization"; Fig. 2 right, first box).
+ *   X      fp16 [T][K] input rows (tokens).
+ *   gamma  fp16 [K] or NULL.  NULL selects quant-only mode: y = x.
+ *   beta   fp16 [K] or NULL (= 0).  Ignored when gamma is NULL.
+ *   eps    LayerNorm epsilon (added to the biased variance).
+ *   Xq     int8 [T][K] output, s_tok fp32 [T] output:
+ *          y = fp16(((x - mean) * rstd) * gamma + beta), mean and biased
+ *          variance computed exactly (integer sums of x*2^24 and its square),
+ *          rstd = fp32(1/sqrt(var + eps)) in fp64;
+ *          s_tok[t] = amax_t/127 with amax_t = max_k |y|,
+ *          Xq = clamp(rne(y * (127/amax_t)), -127, 127); zero rows give 0.
+ *   Y_ln   fp16 [T][K] or NULL: also store y (unfused form, for checking).
+ * Requirements: T >= 0 (T == 0 is a no-op), 16 <= K <= 32768, K % 16 == 0,
+ * pointers 16-byte aligned.
+ */
+zq_status zq_ln_quant(const void* X, const void* gamma, const void* beta, int T, int K, float eps,
+                      int8_t* Xq, float* s_tok, void* Y_ln, zq_stream_t stream);
+
+/*
+ * zq_gemm_w8a8 -- INT8 x INT8 GEMM with the dequantization fused into the
+ * epilogue (Sec. 3.4 "CUTLASS INT8 GEMM" and "Dequantization fused into the
+ * GEMM epilogue"; Fig. 2 right, second box).
+ *   Xq, s_tok   int8 [T][K] and fp32 [T] from zq_ln_quant.
+ *   Wq, s_grp   int8 [N][K] and fp32 [g] from zq_quantize_weights_groupwise.
+ *   bias        fp16 [N] or NULL (= 0).
+ *   Y           fp16 [T][N]:
+ *               acc[t][o] = sum_k Xq[t][k]*Wq[o][k]   (exact, int32)
+ *               Y[t][o] = fp16(((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]))
+ *   acc_dbg     int32 [T][N] or NULL: also store acc (for checking).
+ * Runs on tcgen05 tensor cores.  Small T (weight-streaming) shapes split K
+ * across SMs and reduce the exact int32 partial sums in a library-owned
+ * workspace; calls that use it on different streams must not overlap.
+ * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
+ * 16 <= K <= 133136, K % 16 == 0 (so that 127*127*K < 2^31), 1 <= g <= N,
+ * pointers 16-byte aligned.
+ */
+zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
+                       const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,
+                       int32_t* acc_dbg, zq_stream_t stream);
+
+/*
+ * zq_gemm_w4a8 -- as zq_gemm_w8a8 with INT4 weights (Sec. 3.4 "Which weights
+ * get INT4": FFN weights in INT4).  Wq4 is uint8 [N][K/2] in the layout of
+ * zq_quantize_weights_groupwise(bits=4); the kernel unpacks the nibbles to
+ * int8 in shared memory before each tensor-core MMA.
+ * Requirements as zq_gemm_w8a8, plus K % 32 == 0.
+ */
+zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
+                       const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,
+                       int32_t* acc_dbg, zq_stream_t stream);
+
+/*
+ * zq_device_status -- synchronize `stream`, then read and clear the status
+ * word of the current device.  Returns ZQ_OK, ZQ_ERR_TIMEOUT when a kernel
+ * gave up a bounded wait since the last call (*detail receives the kernel's
+ * wait-site code, may be NULL), or ZQ_ERR_CUDA when synchronization failed.
+ */
+zq_status zq_device_status(zq_stream_t stream, int* detail);
+
+/*
+ * zq_set_option / zq_get_option -- process-wide tuning switches used by
+ * tests and benchmarks to force one kernel variant.  0 always means
+ * "automatic".  Unknown keys return ZQ_ERR_UNSUPPORTED.
+ *   ZQ_OPT_GEMM_PATH   1 = token rows on the MMA M side (prefill tiling),
+ *                      2 = weight rows on the MMA M side (weight streaming).
+ *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256).
+ *   ZQ_OPT_SPLIT_K     number of K splits for path 2 (1 = none).
+ *   ZQ_OPT_MAX_CTAS    cap on the number of CTAs of the GEMM (persistent grid).
+ */
+typedef enum {
+  ZQ_OPT_GEMM_PATH = 1,
+  ZQ_OPT_GEMM_BN = 2,
+  ZQ_OPT_SPLIT_K = 3,
+  ZQ_OPT_MAX_CTAS = 4
+} zq_option;
+zq_status zq_set_option(int key, int value);
+int zq_get_option(int key);
+
+/*
+ * zq_debug_wait_timeout -- launches one CTA that waits on a shared-memory
+ * barrier nothing ever arrives at.  The wait is bounded: after about a
+ * second it records ZQ_ERR_TIMEOUT in the status word and the kernel
+ * returns.  Exists to test the bounded-wait path without a real fault.
+ */
+zq_status zq_debug_wait_timeout(zq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ZQ_H_ */

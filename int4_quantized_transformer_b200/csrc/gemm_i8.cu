@@ -1,0 +1,723 @@
+// gemm_i8.cu -- W8A8 / W4A8 GEMM with the dequantization fused into the
+// epilogue, on Blackwell tcgen05 tensor cores (ZeroQuant, arXiv 2206.01861,
+// Sec. 3.4 "CUTLASS INT8 GEMM", "Dequantization fused into the GEMM
+// epilogue", Fig. 2 right; INT4 FFN weights per "Which weights get INT4").
+//
+// One persistent, warp-specialised kernel serves both regimes the paper
+// distinguishes ("Scheduling for different batch sizes"):
+//
+//  * token rows on the MMA M side (large T, tensor-bound): a 128 x BN tile
+//    of Y per work unit, BN in {128, 192, 256} chosen to fill the 148 SMs;
+//  * weight rows on the MMA M side (small T, weight-streaming, HBM-bound):
+//    128 output features x all tokens (padded to BN in {16..256}) per unit,
+//    with K split across SMs when there are fewer weight tiles than SMs.
+//    Integer partial sums are added exactly (red.add.s32) into a workspace;
+//    the last split of each tile (a per-tile counter) applies the dequant.
+//
+// Warp roles (one CTA per SM):
+//   warp 0     TMA producer: activation and weight tiles, 128-byte K slices,
+//              128B-swizzled, into a STAGES-deep mbarrier ring;
+//   warp 1     TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
+//              N=BN, K=32, int32 accumulators in TMEM (two buffers, so the
+//              epilogue of one unit overlaps the mainloop of the next);
+//   warps 2-5  epilogue: tcgen05.ld of the accumulator, then
+//              y = fp16(((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]));
+//              the scales and bias of a unit are loaded before its
+//              accumulator is ready ("read the two groups of quantization
+//              scales in advance");
+//   warps 6-9  (W4A8 only) unpack: packed signed INT4 weights, staged by TMA,
+//              are sign-extended to int8 and written into the MMA's
+//              128B-swizzled K-major layout in shared memory.
+//
+// Every wait on an mbarrier is bounded (about a second), after which the
+// kernel records the wait site in the device status word and every role
+// leaves its loop; in-flight TMA copies and MMAs are drained before TMEM is
+// released.  No barrier spans several warps inside the role loops, so a
+// warp that gives up cannot strand another one.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "zq_internal.h"
+#include "zq_ptx.cuh"
+
+namespace zq {
+namespace {
+
+constexpr int BM = 128;       // MMA M: rows of a tile = TMEM lanes
+constexpr int BK = 128;       // K bytes per pipeline stage (one swizzle row)
+constexpr int UMMA_K = 32;    // K of one tcgen05.mma kind::i8
+constexpr int kSmemBudget = 220 * 1024;
+
+constexpr int pow2_at_least(int v) {
+  int p = 32;
+  while (p < v) p *= 2;
+  return p;
+}
+
+template <int BN_, bool WROWS_, bool W4_>
+struct Cfg {
+  static constexpr int BN = BN_;
+  static constexpr bool WROWS = WROWS_;  // weight rows on the MMA M side
+  static constexpr bool W4 = W4_;
+  static constexpr int ACT_ROWS = WROWS ? BN : BM;
+  static constexpr int W_ROWS = WROWS ? BM : BN;
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) : 0;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
+  // 32-column loads never leave the allocation.
+  static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
+  static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_STRIDE);
+  static constexpr int NUM_EPI_WARPS = 4;
+  static constexpr int NUM_UNPACK_WARPS = W4 ? 4 : 0;
+  static constexpr int NUM_WARPS = 2 + NUM_EPI_WARPS + NUM_UNPACK_WARPS;
+  static constexpr int NUM_THREADS = 32 * NUM_WARPS;
+  // shared memory carve-up (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_P = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_EPI = OFF_P + STAGES * P_BYTES;           // per-warp scale/bias
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * BN * 2 * 4;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
+  static constexpr int NUM_BARS = 3 * STAGES + 4 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(STAGES >= 2, "not enough shared memory for two stages");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+struct GemmParams {
+  const float* s_tok;
+  const float* s_grp;
+  const __half* bias;
+  __half* Y;
+  int32_t* acc_dbg;
+  int32_t* ws;     // split-K partial sums [T][N] (zero between calls)
+  int* counters;   // split-K arrival counts, [m_tiles*n_tiles*4] (zero between calls)
+  int* status;
+  int T, N, K, g;
+  int m_tiles, n_tiles, k_blocks, splits, kb_per_split, num_units;
+};
+
+struct Unit {
+  int m, n, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, const GemmParams& p) {
+  Unit r;
+  const int split = u % p.splits;
+  const int rest = u / p.splits;
+  r.m = rest % p.m_tiles;
+  r.n = rest / p.m_tiles;
+  r.kb0 = split * p.kb_per_split;
+  r.kb1 = min(p.k_blocks, r.kb0 + p.kb_per_split);
+  return r;
+}
+
+__device__ __forceinline__ int group_of(int o, int N, int g) {
+  return static_cast<int>((static_cast<long long>(o) * g) / N);
+}
+
+// Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, and
+// __syncwarp orders the other lanes' later reads after lane 0's acquire.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* status, int site) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, site) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+// Sign-extend the eight nibbles of w (low nibble first) into eight int8.
+__device__ __forceinline__ void unpack8(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  const uint32_t lo = w & 0x0F0F0F0Fu;         // nibbles 0,2,4,6
+  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // nibbles 1,3,5,7
+  uint32_t a = __byte_perm(lo, hi, 0x5140);    // 0,1,2,3
+  uint32_t b = __byte_perm(lo, hi, 0x7362);    // 4,5,6,7
+  // per byte x in [0,15]: ((x ^ 8) + 0x78) ^ 0x80 == x - 16*(x >= 8), no carries
+  o0 = ((a ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+  o1 = ((b ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  __half2 h = __halves2half2(__float2half_rn(a), __float2half_rn(b));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, 1)
+    gemm_i8_kernel(const __grid_constant__ CUtensorMap map_act,
+                   const __grid_constant__ CUtensorMap map_w, const GemmParams p) {
+  constexpr int BN = C::BN;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sA = smem + C::OFF_A;
+  uint8_t* sB = smem + C::OFF_B;
+  uint8_t* sP = smem + C::OFF_P;
+  float* sEpi = reinterpret_cast<float*>(smem + C::OFF_EPI);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* ready_bar = bars + 2 * STAGES;  // W4: unpacked operand ready
+  uint64_t* tfull_bar = bars + 3 * STAGES;  // [2]
+  uint64_t* tempty_bar = tfull_bar + 2;     // [2]
+  uint64_t* drain_bar = tempty_bar + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int* flag_bcast = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+      mbar_init(&ready_bar[s], C::NUM_UNPACK_WARPS > 0 ? C::NUM_UNPACK_WARPS : 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull_bar[b], 1);
+      mbar_init(&tempty_bar[b], C::NUM_EPI_WARPS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *flag_bcast = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&map_act);
+    tma_prefetch_desc(&map_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_act = l2_policy_evict_last();
+      const uint64_t pol_w = C::WROWS ? l2_policy_evict_first() : l2_policy_evict_last();
+      constexpr uint32_t act_bytes = C::ACT_ROWS * BK;
+      constexpr uint32_t w_bytes = C::W4 ? C::P_BYTES : C::W_ROWS * BK;
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills[STAGES];
+      for (int s = 0; s < STAGES; ++s) fills[s] = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit t = decode_unit(u, p);
+        const int act_row = C::WROWS ? t.n * BN : t.m * BM;
+        const int w_row = C::WROWS ? t.m * BM : t.n * BN;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[stage], act_bytes + w_bytes);
+          uint8_t* act_dst = C::WROWS ? sB + stage * C::B_BYTES : sA + stage * C::A_BYTES;
+          tma_load_2d(act_dst, &map_act, &full_bar[stage], kb * BK, act_row, pol_act);
+          if (C::W4) {
+            tma_load_2d(sP + stage * C::P_BYTES, &map_w, &full_bar[stage], kb * (BK / 2), w_row,
+                        pol_w);
+          } else {
+            uint8_t* w_dst = C::WROWS ? sA + stage * C::A_BYTES : sB + stage * C::B_BYTES;
+            tma_load_2d(w_dst, &map_w, &full_bar[stage], kb * BK, w_row, pol_w);
+          }
+          ++fills[stage];
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Drain: every copy this thread issued must land before the CTA exits.
+      int no_abort = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 9);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_i8(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t tphase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit t = decode_unit(u, p);
+        if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, p.status, 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::ACC_STRIDE);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          uint64_t* rb = C::W4 ? &ready_bar[stage] : &full_bar[stage];
+          if (!mbar_wait(rb, phase, abort_flag, p.status, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t db = make_sw128_desc(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            // advance the start address by k*32 bytes (>>4 = 2k) inside the swizzle row
+            mma_i8(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
+                   idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&tfull_bar[buf]);
+        if (++buf == 2) {
+          buf = 0;
+          tphase ^= 1;
+        }
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      mma_commit(drain_bar);
+      int no_abort = 0;
+      mbar_wait(drain_bar, 0, &no_abort, p.status, 8);
+    }
+  } else if (warp < 2 + C::NUM_EPI_WARPS) {
+    // ------------------------------------------------------ epilogue
+    const int ew = warp - 2;           // epilogue warp index 0..3
+    const int quad = warp & 3;         // TMEM lane quadrant this warp may access
+    const int row_in_tile = quad * 32 + lane;
+    float* colv = sEpi + ew * (2 * BN);  // this warp's per-column scale
+    float* colb = colv + BN;             // ... and bias (token-row tiling)
+    int buf = 0;
+    uint32_t tphase = 0;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+      const Unit t = decode_unit(u, p);
+      // Scales and bias of this unit, fetched before its accumulator is ready.
+      float rscale = 0.0f, rbias = 0.0f;
+      int row_idx;
+      if (C::WROWS) {
+        const int o = t.m * BM + row_in_tile;
+        row_idx = o;
+        if (o < p.N) {
+          rscale = __ldg(p.s_grp + group_of(o, p.N, p.g));
+          rbias = p.bias ? __half2float(p.bias[o]) : 0.0f;
+        }
+        for (int c = lane; c < BN; c += 32) {
+          const int tok = t.n * BN + c;
+          colv[c] = tok < p.T ? __ldg(p.s_tok + tok) : 0.0f;
+        }
+      } else {
+        const int tok = t.m * BM + row_in_tile;
+        row_idx = tok;
+        if (tok < p.T) rscale = __ldg(p.s_tok + tok);
+        for (int c = lane; c < BN; c += 32) {
+          const int o = t.n * BN + c;
+          colv[c] = o < p.N ? __ldg(p.s_grp + group_of(o, p.N, p.g)) : 0.0f;
+          colb[c] = (o < p.N && p.bias) ? __half2float(p.bias[o]) : 0.0f;
+        }
+      }
+      __syncwarp();
+      if (!wait_warp(&tfull_bar[buf], tphase, abort_flag, p.status, 4)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                             static_cast<uint32_t>(buf * C::ACC_STRIDE);
+      const bool split = C::WROWS && p.splits > 1;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t acc[32];
+        tmem_ld_32x32b_x32(t_row + c0, acc);
+        tmem_ld_wait();
+        if (C::WROWS) {
+          // lane = output feature o, columns = tokens
+          const int o = row_idx;
+          if (o < p.N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int tok = t.n * BN + c0 + j;
+              if (c0 + j < BN && tok < p.T) {
+                const int a = static_cast<int>(acc[j]);
+                const size_t idx = static_cast<size_t>(tok) * p.N + o;
+                if (split) {
+                  atomicAdd(p.ws + idx, a);
+                } else {
+                  float v = __fmul_rn(__int2float_rn(a), colv[c0 + j]);
+                  v = __fadd_rn(__fmul_rn(v, rscale), rbias);
+                  p.Y[idx] = __float2half_rn(v);
+                  if (p.acc_dbg) p.acc_dbg[idx] = a;
+                }
+              }
+            }
+          }
+        } else {
+          // lane = token, columns = output features
+          const int tok = row_idx;
+          const int o0 = t.n * BN + c0;
+          if (tok < p.T && o0 < p.N) {
+            uint32_t h[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float v0 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), rscale);
+              float v1 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), rscale);
+              v0 = __fadd_rn(__fmul_rn(v0, colv[c0 + j]), colb[c0 + j]);
+              v1 = __fadd_rn(__fmul_rn(v1, colv[c0 + j + 1]), colb[c0 + j + 1]);
+              h[j / 2] = pack_half2(v0, v1);
+            }
+            __half* yrow = p.Y + static_cast<size_t>(tok) * p.N + o0;
+            int32_t* arow = p.acc_dbg ? p.acc_dbg + static_cast<size_t>(tok) * p.N + o0 : nullptr;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if (o0 + 8 * q < p.N) {  // N % 8 == 0: 8-column chunks are all in or all out
+                reinterpret_cast<uint4*>(yrow)[q] = make_uint4(h[4 * q], h[4 * q + 1],
+                                                               h[4 * q + 2], h[4 * q + 3]);
+                if (arow) {
+                  reinterpret_cast<uint4*>(arow)[2 * q] =
+                      make_uint4(acc[8 * q], acc[8 * q + 1], acc[8 * q + 2], acc[8 * q + 3]);
+                  reinterpret_cast<uint4*>(arow)[2 * q + 1] = make_uint4(
+                      acc[8 * q + 4], acc[8 * q + 5], acc[8 * q + 6], acc[8 * q + 7]);
+                }
+              }
+            }
+          }
+        }
+      }
+      // Release the accumulator buffer to the MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      if (++buf == 2) {
+        buf = 0;
+        tphase ^= 1;
+      }
+      if (split) {
+        // The last of the splits of this tile (per 32-row quadrant) finalises:
+        // exact int32 sums -> dequant -> fp16, and leaves the workspace zero.
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+          int* ctr = p.counters + ((t.n * p.m_tiles + t.m) * 4 + quad);
+          last = (atomicAdd(ctr, 1) == p.splits - 1) ? 1 : 0;
+          if (last) *ctr = 0;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          const int o = row_idx;
+          if (o < p.N) {
+            for (int c = 0; c < BN; ++c) {
+              const int tok = t.n * BN + c;
+              if (tok >= p.T) break;
+              const size_t idx = static_cast<size_t>(tok) * p.N + o;
+              const int a = __ldcg(p.ws + idx);
+              p.ws[idx] = 0;
+              float v = __fmul_rn(__int2float_rn(a), colv[c]);
+              v = __fadd_rn(__fmul_rn(v, rscale), rbias);
+              p.Y[idx] = __float2half_rn(v);
+              if (p.acc_dbg) p.acc_dbg[idx] = a;
+            }
+          }
+        }
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------ INT4 unpack (W4A8)
+    if constexpr (C::W4) {
+      const int ut = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..127
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit t = decode_unit(u, p);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!wait_warp(&full_bar[stage], phase, abort_flag, p.status, 5)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* src = sP + stage * C::P_BYTES;
+          uint8_t* dst = C::WROWS ? sA + stage * C::A_BYTES : sB + stage * C::B_BYTES;
+#pragma unroll 4
+          for (int c = ut; c < C::W_ROWS * 8; c += 128) {
+            const int r = c >> 3, j = c & 7;
+            const uint2 pk = *reinterpret_cast<const uint2*>(src + r * (BK / 2) + j * 8);
+            uint4 o;
+            unpack8(pk.x, o.x, o.y);
+            unpack8(pk.y, o.z, o.w);
+            *reinterpret_cast<uint4*>(dst + r * BK + ((j ^ (r & 7)) << 4)) = o;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ready_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+struct Workspace {
+  int32_t* ws = nullptr;
+  size_t ws_elems = 0;
+  int* counters = nullptr;
+  size_t counter_elems = 0;
+};
+std::mutex g_ws_mu;
+Workspace g_ws[64];
+
+cudaError_t ensure_workspace(size_t elems, size_t counters, cudaStream_t st, Workspace** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  Workspace& w = g_ws[dev];
+  if (w.ws_elems < elems) {
+    if (w.ws) cudaFree(w.ws);
+    w.ws = nullptr;
+    w.ws_elems = 0;
+    e = cudaMalloc(&w.ws, elems * sizeof(int32_t));
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(w.ws, 0, elems * sizeof(int32_t), st);
+    if (e != cudaSuccess) return e;
+    w.ws_elems = elems;
+  }
+  if (w.counter_elems < counters) {
+    if (w.counters) cudaFree(w.counters);
+    w.counters = nullptr;
+    w.counter_elems = 0;
+    e = cudaMalloc(&w.counters, counters * sizeof(int));
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(w.counters, 0, counters * sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    w.counter_elems = counters;
+  }
+  *out = &w;
+  return cudaSuccess;
+}
+
+struct Plan {
+  bool wrows;
+  int bn;
+  int m_tiles, n_tiles, k_blocks, splits, kb_per_split, units;
+  double cost;
+};
+
+int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Wave-aware cost in MMA cycles: ceil(units/SMs) * k-blocks per unit * 2*BN
+// (a 128 x BN x 128 int8 block takes about 2*BN cycles), plus a fixed
+// charge per extra wave and per split-K reduction.
+Plan plan_wrows(int T, int N, int K, int sms, int forced_split) {
+  Plan p{};
+  p.wrows = true;
+  int bn = 16;
+  while (bn < T && bn < 256) bn *= 2;
+  p.bn = bn;
+  p.m_tiles = ceil_div(N, BM);
+  p.n_tiles = ceil_div(T, bn);
+  p.k_blocks = ceil_div(K, BK);
+  const int tiles = p.m_tiles * p.n_tiles;
+  double best = 1e30;
+  int best_s = 1;
+  const int max_s = forced_split > 0 ? forced_split : std::min(p.k_blocks, 32);
+  const int min_s = forced_split > 0 ? forced_split : 1;
+  for (int s = min_s; s <= max_s; ++s) {
+    const int kbps = ceil_div(p.k_blocks, s);
+    const int s_eff = ceil_div(p.k_blocks, kbps);
+    const int units = tiles * s_eff;
+    const int waves = ceil_div(units, sms);
+    // the unit time is set by streaming its weights (HBM-bound): count bytes
+    const double cost = waves * (kbps * 1.0 + 2.0) + (s_eff > 1 ? 1.0 : 0.0);
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_s = s_eff;
+    }
+  }
+  p.kb_per_split = ceil_div(p.k_blocks, best_s);
+  p.splits = ceil_div(p.k_blocks, p.kb_per_split);
+  p.units = tiles * p.splits;
+  p.cost = best * 2.0 * 256;  // comparable scale with the token-row plan
+  return p;
+}
+
+Plan plan_trows(int T, int N, int K, int sms, int forced_bn) {
+  Plan best{};
+  best.cost = 1e30;
+  const int cands[3] = {256, 192, 128};
+  for (int bn : cands) {
+    if (forced_bn && bn != forced_bn) continue;
+    Plan p{};
+    p.wrows = false;
+    p.bn = bn;
+    p.m_tiles = ceil_div(T, BM);
+    p.n_tiles = ceil_div(N, bn);
+    p.k_blocks = ceil_div(K, BK);
+    p.splits = 1;
+    p.kb_per_split = p.k_blocks;
+    p.units = p.m_tiles * p.n_tiles;
+    const int waves = ceil_div(p.units, sms);
+    p.cost = waves * (p.k_blocks * 2.0 * bn + 600.0);
+    if (p.cost < best.cost) best = p;
+  }
+  return best;
+}
+
+template <class C>
+cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const GemmParams& gp,
+                       int grid, cudaStream_t st) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<C>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  gemm_i8_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mw, gp);
+  return cudaGetLastError();
+}
+
+template <bool WROWS, bool W4>
+cudaError_t dispatch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mw,
+                        const GemmParams& gp, int grid, cudaStream_t st) {
+  if constexpr (WROWS) {
+    switch (bn) {
+      case 16: return launch_cfg<Cfg<16, true, W4>>(ma, mw, gp, grid, st);
+      case 32: return launch_cfg<Cfg<32, true, W4>>(ma, mw, gp, grid, st);
+      case 64: return launch_cfg<Cfg<64, true, W4>>(ma, mw, gp, grid, st);
+      case 128: return launch_cfg<Cfg<128, true, W4>>(ma, mw, gp, grid, st);
+      default: return launch_cfg<Cfg<256, true, W4>>(ma, mw, gp, grid, st);
+    }
+  } else {
+    switch (bn) {
+      case 128: return launch_cfg<Cfg<128, false, W4>>(ma, mw, gp, grid, st);
+      case 192: return launch_cfg<Cfg<192, false, W4>>(ma, mw, gp, grid, st);
+      default: return launch_cfg<Cfg<256, false, W4>>(ma, mw, gp, grid, st);
+    }
+  }
+}
+
+zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* Wq,
+                     const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,
+                     int32_t* acc_dbg, zq_stream_t stream) {
+  if (T < 0 || N < 8 || N % 8 != 0 || K < 16 || K % 16 != 0 || K > 133136) return ZQ_ERR_SHAPE;
+  if (w4 && K % 32 != 0) return ZQ_ERR_SHAPE;
+  if (g < 1 || g > N) return ZQ_ERR_SHAPE;
+  if (T == 0) return ZQ_OK;
+  if (!Xq || !s_tok || !Wq || !s_grp || !Y) return ZQ_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (acc_dbg && !aligned16(acc_dbg)))
+    return ZQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+
+  const int forced_path = option(ZQ_OPT_GEMM_PATH);
+  Plan plan;
+  if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
+    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K));
+  } else if (forced_path == 1) {
+    const int fbn = option(ZQ_OPT_GEMM_BN);
+    if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
+    plan = plan_trows(T, N, K, sms, fbn);
+  } else {
+    const Plan a = plan_trows(T, N, K, sms, 0);
+    const Plan b = plan_wrows(T, N, K, sms, 0);
+    plan = b.cost < a.cost ? b : a;
+  }
+
+  int* status = device_status_ptr();
+  if (!status) return ZQ_ERR_CUDA;
+
+  GemmParams gp{};
+  gp.s_tok = s_tok;
+  gp.s_grp = s_grp;
+  gp.bias = static_cast<const __half*>(bias);
+  gp.Y = static_cast<__half*>(Y);
+  gp.acc_dbg = acc_dbg;
+  gp.status = status;
+  gp.T = T;
+  gp.N = N;
+  gp.K = K;
+  gp.g = g;
+  gp.m_tiles = plan.m_tiles;
+  gp.n_tiles = plan.n_tiles;
+  gp.k_blocks = plan.k_blocks;
+  gp.splits = plan.splits;
+  gp.kb_per_split = plan.kb_per_split;
+  gp.num_units = plan.units;
+  if (plan.wrows && plan.splits > 1) {
+    Workspace* w = nullptr;
+    const size_t counters = static_cast<size_t>(plan.m_tiles) * plan.n_tiles * 4;
+    if (ensure_workspace(static_cast<size_t>(T) * N, counters, st, &w) != cudaSuccess)
+      return ZQ_ERR_CUDA;
+    gp.ws = w->ws;
+    gp.counters = w->counters;
+  }
+
+  // TMA descriptors: int8 activations [T][K]; weights int8 [N][K] (128B
+  // swizzle, matching the MMA's K-major layout) or packed int4 [N][K/2]
+  // (plain rows, unpacked into the swizzled layout by the kernel).
+  const int act_rows = plan.wrows ? plan.bn : BM;
+  const int w_rows = plan.wrows ? BM : plan.bn;
+  CUtensorMap ma, mw;
+  if (!encode_tma_2d_u8(&ma, Xq, K, T, K, BK, act_rows, true)) return ZQ_ERR_CUDA;
+  if (w4) {
+    if (!encode_tma_2d_u8(&mw, Wq, K / 2, N, K / 2, BK / 2, w_rows, false)) return ZQ_ERR_CUDA;
+  } else {
+    if (!encode_tma_2d_u8(&mw, Wq, K, N, K, BK, w_rows, true)) return ZQ_ERR_CUDA;
+  }
+
+  int grid = std::min(plan.units, sms);
+  const int cap = option(ZQ_OPT_MAX_CTAS);
+  if (cap > 0) grid = std::min(grid, cap);
+  cudaError_t e;
+  if (plan.wrows)
+    e = w4 ? dispatch_bn<true, true>(plan.bn, ma, mw, gp, grid, st)
+           : dispatch_bn<true, false>(plan.bn, ma, mw, gp, grid, st);
+  else
+    e = w4 ? dispatch_bn<false, true>(plan.bn, ma, mw, gp, grid, st)
+           : dispatch_bn<false, false>(plan.bn, ma, mw, gp, grid, st);
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace zq
+
+extern "C" zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
+                                  const float* s_grp, int g, const void* bias, int T, int N,
+                                  int K, void* Y, int32_t* acc_dbg, zq_stream_t stream) {
+  return zq::gemm_entry(false, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg, stream);
+}
+
+extern "C" zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
+                                  const float* s_grp, int g, const void* bias, int T, int N,
+                                  int K, void* Y, int32_t* acc_dbg, zq_stream_t stream) {
+  return zq::gemm_entry(true, Xq, s_tok, Wq4, s_grp, g, bias, T, N, K, Y, acc_dbg, stream);
+}

@@ -1,0 +1,35 @@
+// zq_internal.h -- declarations shared by the translation units of libzq.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/zq.h"
+
+namespace zq {
+
+// Bounded device-side waits give up after this long (about one second).
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+// Device status word values: 0 = fine; kDevErrTimeoutBase + site = a wait
+// at `site` gave up.
+constexpr int kDevErrTimeoutBase = 1000;
+
+// Device pointer of the current device's status word (set up once per device).
+int* device_status_ptr();
+int num_sms();
+int option(int key);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+// Returns false when the driver entry point is unavailable or encoding fails.
+bool encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                      bool swizzle128);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace zq
+
+#define ZQ_CUDA_OK(expr)                       \
+  do {                                         \
+    if ((expr) != cudaSuccess) return ZQ_ERR_CUDA; \
+  } while (0)

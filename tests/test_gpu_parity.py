@@ -1,0 +1,293 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Integer outputs (int8 codes, packed int4 bytes, int32 accumulators) and the
+fp32 scales must match bit for bit.  fp16 outputs must agree within the
+stated tolerance |y - ref| <= max(1e-3 |ref|, 2 ulp16(ref)); both sides run
+the same IEEE op sequence, so exact equality is expected and asserted too.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int4_quantized_transformer_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def zq():
+    from int4_quantized_transformer_b200 import zq as m
+
+    yield m
+    rc, detail = m.device_status()
+    assert rc == m.ZQ_OK, f"device status {rc} detail {detail}"
+
+
+def dev(t):
+    return t.cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+def ulp16(v):
+    v = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(v, 2.0 ** -14)))
+    return 2.0 ** (e - 10)
+
+
+def assert_fp16_close(y, ref):
+    y64, r64 = y.astype(np.float64), ref.astype(np.float64)
+    tol = np.maximum(1e-3 * np.abs(r64), 2 * ulp16(r64))
+    bad = np.abs(y64 - r64) > tol
+    assert not bad.any(), f"{bad.sum()} fp16 outputs outside tolerance"
+    assert np.array_equal(y.view(np.uint16), ref.view(np.uint16)), \
+        f"{(y.view(np.uint16) != ref.view(np.uint16)).sum()} fp16 outputs differ in the last bits"
+
+
+def assert_bits_equal(a, b):
+    a = np.ascontiguousarray(a)
+    b = np.ascontiguousarray(b)
+    assert a.shape == b.shape
+    av, bv = a.view(np.uint8), b.view(np.uint8)
+    assert np.array_equal(av, bv), f"{(av != bv).sum()} bytes differ"
+
+
+# ------------------------------------------------------------ weights
+
+@pytest.mark.parametrize("N,K,g,bits", [(256, 64, 4, 8), (1024, 1024, 48, 8), (768, 3072, 48, 8),
+                                        (1024, 4096, 64, 4), (96, 64, 7, 4), (64, 32, 64, 4),
+                                        (4096, 4096, 128, 8), (2000, 160, 1, 8)])
+def test_wquant_bit_exact(zq, N, K, g, bits):
+    W = synth.weights(N, K, 0.02, seed=N + K + g)
+    W[: N // 10] *= 8  # unequal group ranges
+    if g > 2:
+        W[N // 2: N // 2 + (N // g)] = 0  # an all-zero stretch of rows
+    qd, sd = zq.quantize_weights_groupwise(dev(W), g, bits)
+    q, s = oracle.quantize_weights_groupwise(W.numpy(), g, bits)
+    if bits == 4:
+        q = oracle.pack_int4(q)
+    assert_bits_equal(host(sd), s)
+    assert_bits_equal(host(qd), q)
+
+
+# ------------------------------------------------------------ ln_quant
+
+@pytest.mark.parametrize("K", [64, 768, 1024, 3072, 4096, 6144, 16384, 24576])
+@pytest.mark.parametrize("mode", ["ln", "ln_no_beta", "quant_only"])
+def test_ln_quant_bit_exact(zq, K, mode):
+    T = 37
+    X = synth.activations(T, K, seed=K, n_outliers=max(1, K // 1000), outlier_scale=30.0)
+    gamma, beta = synth.ln_params(K, K + 1)
+    if mode == "quant_only":
+        gamma = beta = None
+    elif mode == "ln_no_beta":
+        beta = None
+    Xd = dev(X)
+    yd = torch.empty_like(Xd)
+    qd, sd = zq.ln_quant(Xd, None if gamma is None else dev(gamma),
+                         None if beta is None else dev(beta), 1e-5, y_ln=yd)
+    q, s, y = oracle.ln_quant(X.numpy(), None if gamma is None else gamma.numpy(),
+                              None if beta is None else beta.numpy(), 1e-5, want_y=True)
+    assert_bits_equal(host(yd), y)
+    assert_bits_equal(host(sd), s)
+    assert_bits_equal(host(qd), q)
+
+
+@pytest.mark.parametrize("kind", ["zero_rows", "constant_rows", "max_values", "tiny_values"])
+@pytest.mark.parametrize("with_ln", [True, False])
+def test_ln_quant_edge_rows(zq, kind, with_ln):
+    T, K = 29, 768
+    X = synth.edge_activations(kind, T, K)
+    gamma, beta = synth.ln_params(K, 3) if with_ln else (None, None)
+    qd, sd = zq.ln_quant(dev(X), None if gamma is None else dev(gamma),
+                         None if beta is None else dev(beta), 1e-5)
+    q, s = oracle.ln_quant(X.numpy(), None if gamma is None else gamma.numpy(),
+                           None if beta is None else beta.numpy(), 1e-5)
+    assert_bits_equal(host(sd), s)
+    assert_bits_equal(host(qd), q)
+
+
+@pytest.mark.parametrize("T", [1, 2, 9, 1000])
+def test_ln_quant_token_counts(zq, T):
+    K = 1024
+    X = synth.activations(T, K, seed=T, n_outliers=6, outlier_scale=20.0)
+    gamma, beta = synth.ln_params(K, 5)
+    qd, sd = zq.ln_quant(dev(X), dev(gamma), dev(beta), 1e-5)
+    q, s = oracle.ln_quant(X.numpy(), gamma.numpy(), beta.numpy(), 1e-5)
+    assert_bits_equal(host(sd), s)
+    assert_bits_equal(host(qd), q)
+
+
+# ------------------------------------------------------------ GEMM
+
+def _quant_operands(T, N, K, g, bits, seed):
+    X = synth.activations(T, K, seed=seed, n_outliers=6, outlier_scale=20.0)
+    W = synth.weights(N, K, 0.02, seed=seed + 1)
+    b = synth.bias(N, seed + 2)
+    xq, st = oracle.ln_quant(X.numpy())
+    wq, sg = oracle.quantize_weights_groupwise(W.numpy(), g, bits)
+    return xq, st, wq, sg, b.numpy()
+
+
+def _run_gemm(zq, xq, st, wq, sg, b, bits, **opts):
+    T, K = xq.shape
+    N = wq.shape[0]
+    wdev = torch.from_numpy(oracle.pack_int4(wq) if bits == 4 else wq).cuda()
+    acc = torch.empty((T, N), dtype=torch.int32, device="cuda")
+    fn = zq.gemm_w4a8 if bits == 4 else zq.gemm_w8a8
+    with zq.options(**opts):
+        Y = fn(torch.from_numpy(xq).cuda(), torch.from_numpy(st).cuda(), wdev,
+               torch.from_numpy(sg).cuda(), None if b is None else torch.from_numpy(b).cuda(),
+               acc_dbg=acc)
+    return host(Y), host(acc)
+
+
+def _check_gemm(zq, T, N, K, g, bits, seed=0, bias=True, **opts):
+    xq, st, wq, sg, b = _quant_operands(T, N, K, g, bits, seed)
+    if not bias:
+        b = None
+    Y, acc = _run_gemm(zq, xq, st, wq, sg, b, bits, **opts)
+    acc_ref = oracle.gemm_i32(xq, wq)
+    assert_bits_equal(acc, acc_ref)
+    assert_fp16_close(Y, oracle.dequant(acc_ref, st, sg, b))
+
+
+GEMM_SHAPES = [
+    # T, N, K, g
+    (16, 256, 64, 4),      # the single-layer configuration
+    (1, 256, 64, 4),
+    (7, 768, 768, 48),
+    (129, 1024, 768, 48),  # ragged token tile
+    (300, 768, 784, 48),   # K not a multiple of 128
+    (256, 2304, 768, 48),
+    (513, 1000, 256, 3),   # N not a multiple of the tile, N % g != 0
+]
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("T,N,K,g", GEMM_SHAPES)
+def test_gemm_auto(zq, bits, T, N, K, g):
+    if bits == 4 and K % 32:
+        pytest.skip("int4 needs K % 32 == 0")
+    _check_gemm(zq, T, N, K, g, bits, seed=T + N + K)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("bn", [128, 192, 256])
+@pytest.mark.parametrize("T,N,K", [(16, 256, 64), (300, 1000, 512), (1024, 768, 1024)])
+def test_gemm_token_rows_tiles(zq, bits, bn, T, N, K):
+    _check_gemm(zq, T, N, K, 8, bits, seed=bn, path=1, bn=bn)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("split", [1, 2, 3, 7])
+@pytest.mark.parametrize("T,N,K", [(1, 512, 1024), (8, 1024, 896), (64, 384, 2048),
+                                   (200, 256, 1024), (300, 256, 512)])
+def test_gemm_weight_rows_split_k(zq, bits, split, T, N, K):
+    _check_gemm(zq, T, N, K, 16, bits, seed=split, path=2, split_k=split)
+
+
+def test_gemm_persistent_loop_with_few_ctas(zq):
+    # fewer CTAs than work units: every CTA walks several units through both
+    # TMEM accumulator buffers
+    _check_gemm(zq, 640, 1024, 512, 8, 8, seed=3, path=1, bn=128, max_ctas=5)
+    _check_gemm(zq, 640, 1024, 512, 8, 4, seed=4, path=1, bn=256, max_ctas=3)
+    _check_gemm(zq, 16, 2048, 1024, 8, 8, seed=5, path=2, split_k=4, max_ctas=7)
+
+
+def test_gemm_no_bias_and_extremes(zq):
+    # saturated operands: every product is +-127*127 (int8) and accumulators
+    # reach +-127*127*K
+    T, N, K, g = 64, 256, 4096, 2
+    xq = np.full((T, K), 127, np.int8)
+    xq[1::2] = -127
+    wq = np.full((N, K), 127, np.int8)
+    wq[::3] = -127
+    st = np.linspace(1e-3, 1e-2, T).astype(np.float32)
+    sg = np.array([1e-4, 2e-4], np.float32)
+    for bits in (8, 4):
+        w = wq if bits == 8 else np.sign(wq).astype(np.int8) * 7
+        Y, acc = _run_gemm(zq, xq, st, w, sg, None, bits)
+        acc_ref = oracle.gemm_i32(xq, w)
+        assert_bits_equal(acc, acc_ref)
+        assert_fp16_close(Y, oracle.dequant(acc_ref, st, sg, None))
+
+
+def test_gemm_zero_scales_give_bias(zq):
+    T, N, K, g = 5, 64, 128, 4
+    xq, st, wq, sg, b = _quant_operands(T, N, K, g, 8, 11)
+    st[:] = 0
+    Y, _ = _run_gemm(zq, xq, st, wq, sg, b, 8)
+    assert_bits_equal(Y, np.broadcast_to(b, (T, N)))
+
+
+def test_repeated_split_k_calls_leave_workspace_clean(zq):
+    # the split-K workspace must return to zero after every call
+    for i in range(3):
+        _check_gemm(zq, 8, 1024, 2048, 8, 8, seed=100 + i, path=2, split_k=8)
+
+
+# ------------------------------------------------------------ full-size configurations
+
+def _sample_rows(T, n=6):
+    rows = sorted(set([0, T - 1] + list(np.random.default_rng(T).integers(0, T, n))))
+    return np.array(rows)
+
+
+FULL = [(layer, gi, T) for layer in ("bert_base", "gpt350m", "gptj6b", "neox20b")
+        for gi in range(4) for T in synth.LAYERS[layer].tokens]
+
+
+@pytest.mark.parametrize("layer,gi,T", FULL)
+def test_full_size_sampled_rows(zq, layer, gi, T):
+    """Every GEMM of every layer configuration at its full size, in the launch
+    configuration the benchmark uses; the oracle recomputes sampled token
+    rows (each row depends only on its own activations and all weights)."""
+    inp = synth.gemm_inputs(layer, gi, T)
+    s = inp.spec
+    Xd, Wd, bd = dev(inp.X), dev(inp.W), dev(inp.b)
+    gd = None if inp.gamma is None else dev(inp.gamma)
+    betad = None if inp.beta is None else dev(inp.beta)
+    wq_d, sg_d = zq.quantize_weights_groupwise(Wd, s.g, s.bits)
+    xq_d, st_d = zq.ln_quant(Xd, gd, betad, 1e-5)
+    acc_d = torch.empty((T, s.N), dtype=torch.int32, device="cuda")
+    fn = zq.gemm_w4a8 if s.bits == 4 else zq.gemm_w8a8
+    Y_d = fn(xq_d, st_d, wq_d, sg_d, bd, acc_dbg=acc_d)
+
+    wq, sg = oracle.quantize_weights_groupwise(inp.W.numpy(), s.g, s.bits)
+    assert_bits_equal(host(sg_d), sg)
+    assert_bits_equal(host(wq_d), oracle.pack_int4(wq) if s.bits == 4 else wq)
+    rows = _sample_rows(T)
+    Xs = inp.X.numpy()[rows]
+    xq, st = oracle.ln_quant(Xs, None if inp.gamma is None else inp.gamma.numpy(),
+                             None if inp.beta is None else inp.beta.numpy(), 1e-5)
+    assert_bits_equal(host(xq_d)[rows], xq)
+    assert_bits_equal(host(st_d)[rows], st)
+    acc = oracle.gemm_i32(xq, wq)
+    assert_bits_equal(host(acc_d)[rows], acc)
+    assert_fp16_close(host(Y_d)[rows], oracle.dequant(acc, st, sg, inp.b.numpy()))
+
+
+# ------------------------------------------------------------ errors on the device
+
+def test_bounded_wait_reports_timeout(zq):
+    rc, _ = zq.device_status()
+    assert rc == zq.ZQ_OK
+    zq.debug_wait_timeout()
+    rc, detail = zq.device_status()
+    assert rc == zq.ZQ_ERR_TIMEOUT and detail > 0
+    # the context is still usable and the status word was cleared
+    _check_gemm(zq, 16, 256, 64, 4, 8)
+    assert zq.device_status()[0] == zq.ZQ_OK
+
+
+def test_misaligned_device_pointer_rejected(zq):
+    X = torch.zeros(4 * 64 + 8, dtype=torch.float16, device="cuda")
+    Xq = torch.zeros(4 * 64, dtype=torch.int8, device="cuda")
+    s = torch.zeros(4, dtype=torch.float32, device="cuda")
+    rc = zq.lib().zq_ln_quant(X.data_ptr() + 2, None, None, 4, 64, 1e-5, Xq.data_ptr(),
+                              s.data_ptr(), None, None)
+    assert rc == zq.ZQ_ERR_ALIGN

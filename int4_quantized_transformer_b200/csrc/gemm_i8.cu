@@ -20,12 +20,13 @@
 //   warp 1     TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
 //              N=BN, K=32, int32 accumulators in TMEM (two buffers, so the
 //              epilogue of one unit overlaps the mainloop of the next);
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, then
+//   warps 2-9  epilogue, two warps per TMEM lane quadrant, each taking half
+//              of the columns: tcgen05.ld of the accumulator, then
 //              y = fp16(((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]));
 //              the scales and bias of a unit are loaded before its
 //              accumulator is ready ("read the two groups of quantization
 //              scales in advance");
-//   warps 6-9  (W4A8 only) unpack: packed signed INT4 weights, staged by TMA,
+//   warps 10-13 (W4A8 only) unpack: packed signed INT4 weights, staged by TMA,
 //              are sign-extended to int8 and written into the MMA's
 //              128B-swizzled K-major layout in shared memory.
 //
@@ -48,7 +49,8 @@ namespace {
 constexpr int BM = 128;       // MMA M: rows of a tile = TMEM lanes
 constexpr int BK = 128;       // K bytes per pipeline stage (one swizzle row)
 constexpr int UMMA_K = 32;    // K of one tcgen05.mma kind::i8
-constexpr int kSmemBudget = 220 * 1024;
+constexpr int kSmemBudget = 223 * 1024;
+constexpr int NUM_EPI_WARPS_C = 8;
 
 constexpr int pow2_at_least(int v) {
   int p = 32;
@@ -67,13 +69,15 @@ struct Cfg {
   static constexpr int B_BYTES = BN * BK;
   static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) : 0;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
-  static constexpr int STAGES_RAW = kSmemBudget / STAGE_BYTES;
+  static constexpr int STAGES_RAW =
+      (kSmemBudget - (WROWS ? 0 : NUM_EPI_WARPS_C * 32 * 64) - 8 * (BN >= 64 ? BN / 2 : BN) * 8) /
+      STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
   // 32-column loads never leave the allocation.
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
   static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_STRIDE);
-  static constexpr int NUM_EPI_WARPS = 4;
+  static constexpr int NUM_EPI_WARPS = NUM_EPI_WARPS_C;
   static constexpr int NUM_UNPACK_WARPS = W4 ? 4 : 0;
   static constexpr int NUM_WARPS = 2 + NUM_EPI_WARPS + NUM_UNPACK_WARPS;
   static constexpr int NUM_THREADS = 32 * NUM_WARPS;
@@ -81,9 +85,15 @@ struct Cfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_P = OFF_B + STAGES * B_BYTES;
+  // columns handled by one epilogue warp (two warps share a lane quadrant)
+  static constexpr int EPI_COLS = BN >= 64 ? BN / 2 : BN;
   static constexpr int OFF_EPI = OFF_P + STAGES * P_BYTES;           // per-warp scale/bias
-  static constexpr int EPI_BYTES = NUM_EPI_WARPS * BN * 2 * 4;
-  static constexpr int OFF_BAR = OFF_EPI + EPI_BYTES;
+  static constexpr int EPI_BYTES = NUM_EPI_WARPS * EPI_COLS * 2 * 4;
+  // token-row tiling: per-warp staging of a 32 x 32 fp16 output block for
+  // the TMA store (64-byte rows, 64-byte swizzle)
+  static constexpr int STG_BYTES = WROWS ? 0 : 32 * 64;
+  static constexpr int OFF_STG = ((OFF_EPI + EPI_BYTES + 1023) / 1024) * 1024;
+  static constexpr int OFF_BAR = OFF_STG + NUM_EPI_WARPS * STG_BYTES;
   static constexpr int NUM_BARS = 3 * STAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
@@ -98,8 +108,8 @@ struct GemmParams {
   const __half* bias;
   __half* Y;
   int32_t* acc_dbg;
-  int32_t* ws;     // split-K partial sums [T][N] (zero between calls)
-  int* counters;   // split-K arrival counts, [m_tiles*n_tiles*4] (zero between calls)
+  int32_t* ws;     // split-K partial sums [splits][T][N]
+  int* counters;   // split-K arrival counts, [m_tiles*n_tiles*8] (zero between calls)
   int* status;
   int T, N, K, g;
   int m_tiles, n_tiles, k_blocks, splits, kb_per_split, num_units;
@@ -154,7 +164,8 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 template <class C>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     gemm_i8_kernel(const __grid_constant__ CUtensorMap map_act,
-                   const __grid_constant__ CUtensorMap map_w, const GemmParams p) {
+                   const __grid_constant__ CUtensorMap map_w,
+                   const __grid_constant__ CUtensorMap map_y, const GemmParams p) {
   constexpr int BN = C::BN;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -163,6 +174,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   uint8_t* sB = smem + C::OFF_B;
   uint8_t* sP = smem + C::OFF_P;
   float* sEpi = reinterpret_cast<float*>(smem + C::OFF_EPI);
+  uint8_t* sStg = smem + C::OFF_STG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
@@ -193,6 +205,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&map_act);
     tma_prefetch_desc(&map_w);
+    if (!C::WROWS) tma_prefetch_desc(&map_y);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -207,7 +220,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_act = l2_policy_evict_last();
-      const uint64_t pol_w = C::WROWS ? l2_policy_evict_first() : l2_policy_evict_last();
+      // weights: streamed once when weight rows are the M side; in the
+      // token-row tiling they are re-read by every token tile but can be far
+      // larger than L2, so they get the first-to-go policy only in the former.
+      const uint64_t pol_w = C::WROWS ? l2_policy_evict_first() : l2_policy_evict_normal();
       constexpr uint32_t act_bytes = C::ACT_ROWS * BK;
       constexpr uint32_t w_bytes = C::W4 ? C::P_BYTES : C::W_ROWS * BK;
       int stage = 0;
@@ -295,11 +311,19 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
   } else if (warp < 2 + C::NUM_EPI_WARPS) {
     // ------------------------------------------------------ epilogue
-    const int ew = warp - 2;           // epilogue warp index 0..3
-    const int quad = warp & 3;         // TMEM lane quadrant this warp may access
+    // Two warps per TMEM lane quadrant (a warp may only read the 32 lanes of
+    // quadrant warp%4); each takes half of the tile's columns.
+    const int ew = warp - 2;          // epilogue warp index 0..7
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
+    const int half = ew >> 2;         // which half of the columns
     const int row_in_tile = quad * 32 + lane;
-    float* colv = sEpi + ew * (2 * BN);  // this warp's per-column scale
-    float* colb = colv + BN;             // ... and bias (token-row tiling)
+    constexpr bool kSplitCols = BN >= 64;
+    const int cb = kSplitCols ? half * (BN / 2) : 0;                       // first column
+    const int ce = kSplitCols ? cb + BN / 2 : (half == 0 ? BN : 0);        // one past the last
+    // this warp's per-column scale and bias, indexed from its first column cb
+    float* colv = sEpi + ew * (2 * C::EPI_COLS) - cb;
+    float* colb = colv + C::EPI_COLS;
+    uint8_t* stg = sStg + ew * C::STG_BYTES;
     int buf = 0;
     uint32_t tphase = 0;
     for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
@@ -314,7 +338,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           rscale = __ldg(p.s_grp + group_of(o, p.N, p.g));
           rbias = p.bias ? __half2float(p.bias[o]) : 0.0f;
         }
-        for (int c = lane; c < BN; c += 32) {
+        for (int c = cb + lane; c < ce; c += 32) {
           const int tok = t.n * BN + c;
           colv[c] = tok < p.T ? __ldg(p.s_tok + tok) : 0.0f;
         }
@@ -322,7 +346,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         const int tok = t.m * BM + row_in_tile;
         row_idx = tok;
         if (tok < p.T) rscale = __ldg(p.s_tok + tok);
-        for (int c = lane; c < BN; c += 32) {
+        for (int c = cb + lane; c < ce; c += 32) {
           const int o = t.n * BN + c;
           colv[c] = o < p.N ? __ldg(p.s_grp + group_of(o, p.N, p.g)) : 0.0f;
           colb[c] = (o < p.N && p.bias) ? __half2float(p.bias[o]) : 0.0f;
@@ -334,11 +358,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(buf * C::ACC_STRIDE);
       const bool split = C::WROWS && p.splits > 1;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t acc[32];
-        tmem_ld_32x32b_x32(t_row + c0, acc);
-        tmem_ld_wait();
+
+      auto process = [&](const uint32_t (&acc)[32], int c0) {
         if (C::WROWS) {
           // lane = output feature o, columns = tokens
           const int o = row_idx;
@@ -350,7 +371,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
                 const int a = static_cast<int>(acc[j]);
                 const size_t idx = static_cast<size_t>(tok) * p.N + o;
                 if (split) {
-                  atomicAdd(p.ws + idx, a);
+                  p.ws[static_cast<size_t>(t.kb0 / p.kb_per_split) * p.T * p.N + idx] = a;
                 } else {
                   float v = __fmul_rn(__int2float_rn(a), colv[c0 + j]);
                   v = __fadd_rn(__fmul_rn(v, rscale), rbias);
@@ -364,24 +385,28 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           // lane = token, columns = output features
           const int tok = row_idx;
           const int o0 = t.n * BN + c0;
+          uint32_t h[16];
           if (tok < p.T && o0 < p.N) {
-            uint32_t h[16];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
+            for (int j = 0; j < 32; j += 4) {
+              const float4 sv = *reinterpret_cast<const float4*>(colv + c0 + j);
+              const float4 bv = *reinterpret_cast<const float4*>(colb + c0 + j);
               float v0 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), rscale);
               float v1 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), rscale);
-              v0 = __fadd_rn(__fmul_rn(v0, colv[c0 + j]), colb[c0 + j]);
-              v1 = __fadd_rn(__fmul_rn(v1, colv[c0 + j + 1]), colb[c0 + j + 1]);
+              float v2 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 2])), rscale);
+              float v3 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 3])), rscale);
+              v0 = __fadd_rn(__fmul_rn(v0, sv.x), bv.x);
+              v1 = __fadd_rn(__fmul_rn(v1, sv.y), bv.y);
+              v2 = __fadd_rn(__fmul_rn(v2, sv.z), bv.z);
+              v3 = __fadd_rn(__fmul_rn(v3, sv.w), bv.w);
               h[j / 2] = pack_half2(v0, v1);
+              h[j / 2 + 1] = pack_half2(v2, v3);
             }
-            __half* yrow = p.Y + static_cast<size_t>(tok) * p.N + o0;
             int32_t* arow = p.acc_dbg ? p.acc_dbg + static_cast<size_t>(tok) * p.N + o0 : nullptr;
+            if (arow) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              if (o0 + 8 * q < p.N) {  // N % 8 == 0: 8-column chunks are all in or all out
-                reinterpret_cast<uint4*>(yrow)[q] = make_uint4(h[4 * q], h[4 * q + 1],
-                                                               h[4 * q + 2], h[4 * q + 3]);
-                if (arow) {
+              for (int q = 0; q < 4; ++q) {
+                if (o0 + 8 * q < p.N) {  // N % 8 == 0: 8-column chunks are all in or all out
                   reinterpret_cast<uint4*>(arow)[2 * q] =
                       make_uint4(acc[8 * q], acc[8 * q + 1], acc[8 * q + 2], acc[8 * q + 3]);
                   reinterpret_cast<uint4*>(arow)[2 * q + 1] = make_uint4(
@@ -390,7 +415,38 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
               }
             }
           }
+          // The warp's 32 rows x 32 columns go out as one TMA tensor store
+          // (rows past T / columns past N are clipped by the TMA unit): wait
+          // until the previous store has read the staging buffer, write this
+          // lane's 64-byte row in the 64B-swizzled layout, then issue.
+          if (o0 < p.N && t.m * BM + quad * 32 < p.T) {  // warp-uniform
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ sw) << 4)) =
+                  make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&map_y, stg, o0, t.m * BM + quad * 32);
+              bulk_commit_group();
+            }
+          }
         }
+      };
+
+      // Two 32-column TMEM loads in flight before each wait.
+#pragma unroll 1
+      for (int c0 = cb; c0 < ce; c0 += 64) {
+        uint32_t a0[32], a1[32];
+        const bool two = c0 + 32 < ce;
+        tmem_ld_32x32b_x32(t_row + c0, a0);
+        if (two) tmem_ld_32x32b_x32(t_row + c0 + 32, a1);
+        tmem_ld_wait();
+        process(a0, c0);
+        if (two) process(a1, c0 + 32);
       }
       // Release the accumulator buffer to the MMA warp.
       tc_fence_before();
@@ -400,14 +456,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         buf = 0;
         tphase ^= 1;
       }
-      if (split) {
-        // The last of the splits of this tile (per 32-row quadrant) finalises:
-        // exact int32 sums -> dequant -> fp16, and leaves the workspace zero.
+      if (split && cb < ce) {
+        // The last of the splits of this tile finalises its (quadrant, column
+        // half): the exact int32 partial sums of all splits -> dequant -> fp16.
         __threadfence();
         __syncwarp();
         int last = 0;
         if (lane == 0) {
-          int* ctr = p.counters + ((t.n * p.m_tiles + t.m) * 4 + quad);
+          int* ctr = p.counters + (((t.n * p.m_tiles + t.m) * 4 + quad) * 2 + half);
           last = (atomicAdd(ctr, 1) == p.splits - 1) ? 1 : 0;
           if (last) *ctr = 0;
         }
@@ -416,12 +472,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           __threadfence();
           const int o = row_idx;
           if (o < p.N) {
-            for (int c = 0; c < BN; ++c) {
+            for (int c = cb; c < ce; ++c) {
               const int tok = t.n * BN + c;
               if (tok >= p.T) break;
               const size_t idx = static_cast<size_t>(tok) * p.N + o;
-              const int a = __ldcg(p.ws + idx);
-              p.ws[idx] = 0;
+              const size_t plane = static_cast<size_t>(p.T) * p.N;
+              int a = 0;
+              for (int sp = 0; sp < p.splits; ++sp) a += __ldcg(p.ws + sp * plane + idx);
               float v = __fmul_rn(__int2float_rn(a), colv[c]);
               v = __fadd_rn(__fmul_rn(v, rscale), rbias);
               p.Y[idx] = __float2half_rn(v);
@@ -469,6 +526,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
   }
 
+  if (!C::WROWS && warp >= 2 && warp < 2 + C::NUM_EPI_WARPS && lane == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -588,8 +646,8 @@ Plan plan_trows(int T, int N, int K, int sms, int forced_bn) {
 }
 
 template <class C>
-cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const GemmParams& gp,
-                       int grid, cudaStream_t st) {
+cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& my,
+                       const GemmParams& gp, int grid, cudaStream_t st) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -600,26 +658,26 @@ cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const GemmP
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  gemm_i8_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mw, gp);
+  gemm_i8_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mw, my, gp);
   return cudaGetLastError();
 }
 
 template <bool WROWS, bool W4>
 cudaError_t dispatch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mw,
-                        const GemmParams& gp, int grid, cudaStream_t st) {
+                        const CUtensorMap& my, const GemmParams& gp, int grid, cudaStream_t st) {
   if constexpr (WROWS) {
     switch (bn) {
-      case 16: return launch_cfg<Cfg<16, true, W4>>(ma, mw, gp, grid, st);
-      case 32: return launch_cfg<Cfg<32, true, W4>>(ma, mw, gp, grid, st);
-      case 64: return launch_cfg<Cfg<64, true, W4>>(ma, mw, gp, grid, st);
-      case 128: return launch_cfg<Cfg<128, true, W4>>(ma, mw, gp, grid, st);
-      default: return launch_cfg<Cfg<256, true, W4>>(ma, mw, gp, grid, st);
+      case 16: return launch_cfg<Cfg<16, true, W4>>(ma, mw, my, gp, grid, st);
+      case 32: return launch_cfg<Cfg<32, true, W4>>(ma, mw, my, gp, grid, st);
+      case 64: return launch_cfg<Cfg<64, true, W4>>(ma, mw, my, gp, grid, st);
+      case 128: return launch_cfg<Cfg<128, true, W4>>(ma, mw, my, gp, grid, st);
+      default: return launch_cfg<Cfg<256, true, W4>>(ma, mw, my, gp, grid, st);
     }
   } else {
     switch (bn) {
-      case 128: return launch_cfg<Cfg<128, false, W4>>(ma, mw, gp, grid, st);
-      case 192: return launch_cfg<Cfg<192, false, W4>>(ma, mw, gp, grid, st);
-      default: return launch_cfg<Cfg<256, false, W4>>(ma, mw, gp, grid, st);
+      case 128: return launch_cfg<Cfg<128, false, W4>>(ma, mw, my, gp, grid, st);
+      case 192: return launch_cfg<Cfg<192, false, W4>>(ma, mw, my, gp, grid, st);
+      default: return launch_cfg<Cfg<256, false, W4>>(ma, mw, my, gp, grid, st);
     }
   }
 }
@@ -638,18 +696,16 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int sms = num_sms();
 
+  // Weight rows on the MMA M side for small token counts (weight streaming),
+  // token rows otherwise; tests and benchmarks may force either.
   const int forced_path = option(ZQ_OPT_GEMM_PATH);
   Plan plan;
   if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
     plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K));
-  } else if (forced_path == 1) {
+  } else {
     const int fbn = option(ZQ_OPT_GEMM_BN);
     if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
     plan = plan_trows(T, N, K, sms, fbn);
-  } else {
-    const Plan a = plan_trows(T, N, K, sms, 0);
-    const Plan b = plan_wrows(T, N, K, sms, 0);
-    plan = b.cost < a.cost ? b : a;
   }
 
   int* status = device_status_ptr();
@@ -674,8 +730,8 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   gp.num_units = plan.units;
   if (plan.wrows && plan.splits > 1) {
     Workspace* w = nullptr;
-    const size_t counters = static_cast<size_t>(plan.m_tiles) * plan.n_tiles * 4;
-    if (ensure_workspace(static_cast<size_t>(T) * N, counters, st, &w) != cudaSuccess)
+    const size_t counters = static_cast<size_t>(plan.m_tiles) * plan.n_tiles * 8;
+    if (ensure_workspace(static_cast<size_t>(plan.splits) * T * N, counters, st, &w) != cudaSuccess)
       return ZQ_ERR_CUDA;
     gp.ws = w->ws;
     gp.counters = w->counters;
@@ -686,24 +742,34 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   // (plain rows, unpacked into the swizzled layout by the kernel).
   const int act_rows = plan.wrows ? plan.bn : BM;
   const int w_rows = plan.wrows ? BM : plan.bn;
-  CUtensorMap ma, mw;
-  if (!encode_tma_2d_u8(&ma, Xq, K, T, K, BK, act_rows, true)) return ZQ_ERR_CUDA;
+  CUtensorMap ma, mw, my;
+  if (!encode_tma_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, T, K, BK, act_rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return ZQ_ERR_CUDA;
   if (w4) {
-    if (!encode_tma_2d_u8(&mw, Wq, K / 2, N, K / 2, BK / 2, w_rows, false)) return ZQ_ERR_CUDA;
+    if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K / 2, N, K / 2, BK / 2, w_rows,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))
+      return ZQ_ERR_CUDA;
   } else {
-    if (!encode_tma_2d_u8(&mw, Wq, K, N, K, BK, w_rows, true)) return ZQ_ERR_CUDA;
+    if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, BK, w_rows,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+      return ZQ_ERR_CUDA;
   }
+  // fp16 output [T][N]: 32 x 32 boxes written by the epilogue warps
+  if (!encode_tma_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
+                     32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return ZQ_ERR_CUDA;
 
   int grid = std::min(plan.units, sms);
   const int cap = option(ZQ_OPT_MAX_CTAS);
   if (cap > 0) grid = std::min(grid, cap);
   cudaError_t e;
   if (plan.wrows)
-    e = w4 ? dispatch_bn<true, true>(plan.bn, ma, mw, gp, grid, st)
-           : dispatch_bn<true, false>(plan.bn, ma, mw, gp, grid, st);
+    e = w4 ? dispatch_bn<true, true>(plan.bn, ma, mw, my, gp, grid, st)
+           : dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st);
   else
-    e = w4 ? dispatch_bn<false, true>(plan.bn, ma, mw, gp, grid, st)
-           : dispatch_bn<false, false>(plan.bn, ma, mw, gp, grid, st);
+    e = w4 ? dispatch_bn<false, true>(plan.bn, ma, mw, my, gp, grid, st)
+           : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 

@@ -48,16 +48,32 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 // --------------------------------------------------------------- ln_quant
 
 struct RowSums {
-  long long s1;             // sum of a = x * 2^24
-  unsigned long long p, q, r;  // a^2 = p*2^40 + q*2^21 + r, split |a| = ah*2^20 + al
+  long long s1;                // sum of a = x * 2^24 (an integer for every finite fp16 x)
+  unsigned long long p, q, r;  // sum of a^2 = p*2^40 + q*2^21 + r, with |a| = ah*2^20 + al
 };
 
-__device__ __forceinline__ void add_exact(RowSums& s, float f) {
-  long long a = __float2ll_rz(__fmul_rn(f, 16777216.0f));  // exact: |a| < 2^40
-  s.s1 += a;
-  unsigned long long ua = static_cast<unsigned long long>(a < 0 ? -a : a);
-  uint32_t ah = static_cast<uint32_t>(ua >> 20);
-  uint32_t al = static_cast<uint32_t>(ua) & 0xFFFFFu;
+// Per-thread partial sums, kept in 32-bit where that is exact: a thread adds
+// at most 32 elements, so sum(+-ah) and sum(+-al) stay below 2^26.
+struct ThreadSums {
+  int s1h, s1l;
+  unsigned long long p, q, r;
+};
+
+// Adds one fp16 value x (already converted to fp32, exactly) to the exact
+// sums.  |a| = |x|*2^24 = ah*2^20 + al with ah = floor(|x|*16) and
+// al = frac(|x|*16)*2^20, both below 2^20.  The integer and fractional parts
+// come from the fp32 "magic number" technique: adding 2^23 with rounding
+// toward zero leaves floor(v) in the low mantissa bits of the sum (v < 2^20),
+// and the remaining fraction is an exact multiple of 2^-20.
+__device__ __forceinline__ void add_exact(ThreadSums& s, float x) {
+  const float v = __fmul_rn(fabsf(x), 16.0f);               // |x|*16 < 2^20, exact
+  const float t = __fadd_rz(v, 8388608.0f);                 // 2^23 + floor(v)
+  const uint32_t ah = __float_as_uint(t) - 0x4B000000u;
+  const float fr = __fsub_rn(v, __fsub_rn(t, 8388608.0f));  // v - floor(v), exact
+  const uint32_t al = __float_as_uint(__fmaf_rn(fr, 1048576.0f, 8388608.0f)) - 0x4B000000u;
+  const int sg = (__float_as_int(x) >> 31) | 1;             // -1 or +1
+  s.s1h += sg * static_cast<int>(ah);
+  s.s1l += sg * static_cast<int>(al);
   s.p += static_cast<unsigned long long>(ah) * ah;
   s.q += static_cast<unsigned long long>(ah) * al;
   s.r += static_cast<unsigned long long>(al) * al;
@@ -79,34 +95,37 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// mean and rstd from the exact sums: mean = S1*2^-24/K, E[x^2] = S2*2^-48/K,
-// var = max(E[x^2] - mean^2, 0) (biased), rstd = fp32(1/sqrt(var + eps)).
-__device__ __forceinline__ void row_stats(const RowSums& s, int K, float eps, float& mean,
-                                          float& rstd) {
-  unsigned __int128 s2 = (static_cast<unsigned __int128>(s.p) << 40) +
-                         (static_cast<unsigned __int128>(s.q) << 21) +
-                         static_cast<unsigned __int128>(s.r);
-  unsigned long long hi = static_cast<unsigned long long>(s2 >> 64);
-  unsigned long long lo = static_cast<unsigned long long>(s2);
-  double dk = static_cast<double>(K);
-  double mean_d = __ddiv_rn(__dmul_rn(__ll2double_rn(s.s1), 0x1p-24), dk);
-  double e2 = __dadd_rn(__dmul_rn(__ull2double_rn(hi), 0x1p64), __ull2double_rn(lo));
-  e2 = __ddiv_rn(__dmul_rn(e2, 0x1p-48), dk);
+// mean and rstd from the exact sums, c1 = 2^-24/K and c2 = 2^-48/K (fp64,
+// computed on the host): mean = S1*c1, E[x^2] = S2*c2 with S2 taken to
+// fp64 as hi*2^64 + lo, var = max(E[x^2] - mean^2, 0) (biased) in fp64, then
+// rstd = 1/sqrt(fp32(var) + eps) in fp32.
+__device__ __forceinline__ void row_stats(const RowSums& s, double c1, double c2, float eps,
+                                          float& mean, float& rstd) {
+  const unsigned __int128 s2 = (static_cast<unsigned __int128>(s.p) << 40) +
+                               (static_cast<unsigned __int128>(s.q) << 21) +
+                               static_cast<unsigned __int128>(s.r);
+  const unsigned long long hi = static_cast<unsigned long long>(s2 >> 64);
+  const unsigned long long lo = static_cast<unsigned long long>(s2);
+  const double mean_d = __dmul_rn(__ll2double_rn(s.s1), c1);
+  const double e2 =
+      __dmul_rn(__dadd_rn(__dmul_rn(__ull2double_rn(hi), 0x1p64), __ull2double_rn(lo)), c2);
   double var = __dsub_rn(e2, __dmul_rn(mean_d, mean_d));
   if (var < 0.0) var = 0.0;
-  double denom = __dsqrt_rn(__dadd_rn(var, static_cast<double>(eps)));
-  rstd = __double2float_rn(__ddiv_rn(1.0, denom));
+  const float r = __fsqrt_rn(__fadd_rn(__double2float_rn(var), eps));
+  rstd = __fdiv_rn(1.0f, r);
   mean = __double2float_rn(mean_d);
 }
 
 // W warps per row, VPT 16-byte vectors (8 halves) per thread.  Blocks hold
 // RPB = max(1, 8/W) rows; every thread runs the same number of row
-// iterations so block-wide barriers stay uniform.
+// iterations so block-wide barriers stay uniform.  gamma/beta are re-read
+// per row (they stay in L1) to keep registers low and occupancy high.
 template <int W, int VPT>
-__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
+__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 32) : 8) / 2)
     ln_quant_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
-                    const __half* __restrict__ beta, int T, int K, float eps,
-                    int8_t* __restrict__ Xq, float* __restrict__ s_tok, __half* __restrict__ Y_ln) {
+                    const __half* __restrict__ beta, int T, int K, float eps, double c1,
+                    double c2, int8_t* __restrict__ Xq, float* __restrict__ s_tok,
+                    __half* __restrict__ Y_ln) {
   constexpr int RT = 32 * W;                // threads per row
   constexpr int RPB = W >= 8 ? 1 : 8 / W;   // rows per block
   __shared__ RowSums red_s[RPB][W];
@@ -118,20 +137,6 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
   const int lane = threadIdx.x & 31;
   const int nvec = K / 8;
   const bool ln = gamma != nullptr;
-
-  uint4 g4[VPT], b4[VPT];
-  if (ln) {
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      int v = j + i * RT;
-      g4[i] = make_uint4(0, 0, 0, 0);
-      b4[i] = make_uint4(0, 0, 0, 0);
-      if (v < nvec) {
-        g4[i] = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
-        if (beta) b4[i] = __ldg(reinterpret_cast<const uint4*>(beta) + v);
-      }
-    }
-  }
 
   const int rows_per_iter = gridDim.x * RPB;
   const int iters = (T + rows_per_iter - 1) / rows_per_iter;
@@ -149,13 +154,22 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
     }
 
     if (ln) {
-      RowSums s = {0, 0, 0, 0};
+      ThreadSums ts = {0, 0, 0, 0, 0};
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
-        const __half* h = reinterpret_cast<const __half*>(&x4[i]);
+        const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) add_exact(s, __half2float(h[e]));
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(h[e]);
+          add_exact(ts, f.x);
+          add_exact(ts, f.y);
+        }
       }
+      RowSums s;
+      s.s1 = static_cast<long long>(ts.s1h) * 1048576 + ts.s1l;
+      s.p = ts.p;
+      s.q = ts.q;
+      s.r = ts.r;
       warp_sum(s);
       if (W > 1) {
         if (lane == 0) red_s[slot][warp_in_row] = s;
@@ -170,30 +184,42 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
           s.r += t.r;
         }
       }
-      float mean, rstd;
-      row_stats(s, K, eps, mean, rstd);
+      // One lane does the fp64 row arithmetic; the warp gets it by shuffle.
+      float mean = 0.0f, rstd = 0.0f;
+      if (lane == 0) row_stats(s, c1, c2, eps, mean, rstd);
+      mean = __shfl_sync(0xffffffffu, mean, 0);
+      rstd = __shfl_sync(0xffffffffu, rstd, 0);
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
-        __half* h = reinterpret_cast<__half*>(&x4[i]);
-        const __half* gm = reinterpret_cast<const __half*>(&g4[i]);
-        const __half* bt = reinterpret_cast<const __half*>(&b4[i]);
+        const int v = j + i * RT;
+        if (v < nvec) {
+          const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
+          const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v)
+                                : make_uint4(0, 0, 0, 0);
+          __half2* h = reinterpret_cast<__half2*>(&x4[i]);
+          const __half2* gm = reinterpret_cast<const __half2*>(&g4);
+          const __half2* bt = reinterpret_cast<const __half2*>(&b4);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float d = __fsub_rn(__half2float(h[e]), mean);
-          float n = __fmul_rn(d, rstd);
-          float sc = __fmul_rn(n, __half2float(gm[e]));
-          h[e] = __float2half_rn(__fadd_rn(sc, __half2float(bt[e])));
+          for (int e = 0; e < 4; ++e) {
+            const float2 xf = __half22float2(h[e]);
+            const float2 gf = __half22float2(gm[e]);
+            const float2 bf = __half22float2(bt[e]);
+            const float y0 = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(xf.x, mean), rstd), gf.x), bf.x);
+            const float y1 = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(xf.y, mean), rstd), gf.y), bf.y);
+            h[e] = __halves2half2(__float2half_rn(y0), __float2half_rn(y1));
+          }
         }
       }
     }
 
-    float amax = 0.0f;
+    __half2 m2 = __float2half2_rn(0.0f);
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const __half* h = reinterpret_cast<const __half*>(&x4[i]);
+      const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(__half2float(h[e])));
+      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h[e]));
     }
+    float amax = fmaxf(__low2float(m2), __high2float(m2));
     amax = warp_max(amax);
     if (W > 1) {
       if (lane == 0) red_m[slot][warp_in_row] = amax;
@@ -210,10 +236,14 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
       for (int i = 0; i < VPT; ++i) {
         int v = j + i * RT;
         if (v < nvec) {
-          const __half* h = reinterpret_cast<const __half*>(&x4[i]);
+          const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
           uint32_t c[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) c[e] = quant_code(__half2float(h[e]), inv, 127.0f);
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h[e]);
+            c[2 * e] = quant_code(f.x, inv, 127.0f);
+            c[2 * e + 1] = quant_code(f.y, inv, 127.0f);
+          }
           uint2 out;
           out.x = pack4(c[0], c[1], c[2], c[3]);
           out.y = pack4(c[4], c[5], c[6], c[7]);
@@ -238,7 +268,9 @@ cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, int T, 
   int need = (T + RPB - 1) / RPB;
   int grid = num_sms() * per_sm;
   if (grid > need) grid = need;
-  ln_quant_kernel<W, VPT><<<grid, threads, 0, st>>>(X, g, b, T, K, eps, Xq, s, Y);
+  const double c1 = 0x1p-24 / static_cast<double>(K);
+  const double c2 = 0x1p-48 / static_cast<double>(K);
+  ln_quant_kernel<W, VPT><<<grid, threads, 0, st>>>(X, g, b, T, K, eps, c1, c2, Xq, s, Y);
   return cudaGetLastError();
 }
 

@@ -4,7 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/zq.h"
+#include "zq.h"
 
 namespace zq {
 
@@ -21,9 +21,9 @@ int option(int key);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 // Returns false when the driver entry point is unavailable or encoding fails.
-bool encode_tma_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                      bool swizzle128);
+bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                   uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

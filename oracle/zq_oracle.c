@@ -23,7 +23,9 @@
  *   R2 Clamp to [-qmax, qmax] (qmax = 127 or 7): symmetric, and the absmax
  *      scale never produces -128/-8 anyway.
  *   R3 LayerNorm statistics are computed exactly (integer sums of x*2^24 and
- *      of its square), so they do not depend on summation order.
+ *      of its square), so they do not depend on summation order; mean and
+ *      variance are then formed in fp64 and 1/sqrt(var + eps) in fp32
+ *      (see zqo_ln_row_stats for the exact sequence of roundings).
  *   R4 The fused kernel quantizes its fp16 LayerNorm output (Fig. 2: fused and
  *      unfused compute the same output).
  *   R5 Scales are fp32.
@@ -167,19 +169,26 @@ void zqo_ln_exact_sums(const uint16_t *x, int K, int64_t *S1, uint64_t *S2_hi, u
     *S2_lo = (uint64_t)s2;
 }
 
-/* mean and rstd of one row, from the exact sums (biased variance, /K). */
+/* mean and rstd of one row, from the exact sums (biased variance, /K):
+ *   c1 = 2^-24/K, c2 = 2^-48/K                      (fp64 divisions)
+ *   mean_d = S1*c1, E2 = (hi*2^64 + lo)*c2           (fp64)
+ *   var_d  = max(E2 - mean_d^2, 0)                   (fp64)
+ *   rstd   = 1/sqrt(fp32(var_d) + eps)               (fp32), mean = fp32(mean_d). */
 void zqo_ln_row_stats(const uint16_t *x, int K, float eps, float *mean_out, float *rstd_out,
                       double *mean_d_out, double *var_d_out) {
     int64_t S1;
     uint64_t hi, lo;
     zqo_ln_exact_sums(x, K, &S1, &hi, &lo);
-    double mean_d = ((double)S1 * 0x1p-24) / (double)K;
-    double e2_d = (((double)hi * 0x1p64 + (double)lo) * 0x1p-48) / (double)K;
+    double c1 = 0x1p-24 / (double)K;
+    double c2 = 0x1p-48 / (double)K;
+    double mean_d = (double)S1 * c1;
+    double e2_d = ((double)hi * 0x1p64 + (double)lo) * c2;
     double msq = mean_d * mean_d;
     double var_d = e2_d - msq;
     if (var_d < 0.0) var_d = 0.0;
-    double denom = sqrt(var_d + (double)eps);
-    *rstd_out = (float)(1.0 / denom);
+    float vf = (float)var_d;
+    float r = sqrtf(vf + eps);
+    *rstd_out = 1.0f / r;
     *mean_out = (float)mean_d;
     if (mean_d_out) *mean_d_out = mean_d;
     if (var_d_out) *var_d_out = var_d;

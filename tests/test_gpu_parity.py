@@ -291,3 +291,38 @@ def test_misaligned_device_pointer_rejected(zq):
     rc = zq.lib().zq_ln_quant(X.data_ptr() + 2, None, None, 4, 64, 1e-5, Xq.data_ptr(),
                               s.data_ptr(), None, None)
     assert rc == zq.ZQ_ERR_ALIGN
+
+
+def test_cuda_graph_replay_matches_eager(zq):
+    """The hot path can be recorded once as a CUDA graph and replayed (the
+    paper uses CUDA Graphs for small models); replay gives identical bits."""
+    T, K, N, g = 512, 768, 768, 48
+    X = synth.activations(T, K, seed=21, n_outliers=6, outlier_scale=20.0).cuda()
+    gamma, beta = (t.cuda() for t in synth.ln_params(K, 22))
+    W = synth.weights(N, K, 0.02, seed=23).cuda()
+    b = synth.bias(N, 24).cuda()
+    outs = {}
+    for bits in (8, 4):
+        Wq, sg = zq.quantize_weights_groupwise(W, g, bits)
+        Xq = torch.empty((T, K), dtype=torch.int8, device="cuda")
+        st = torch.empty(T, dtype=torch.float32, device="cuda")
+        Y = torch.empty((T, N), dtype=torch.float16, device="cuda")
+        fn = zq.gemm_w4a8 if bits == 4 else zq.gemm_w8a8
+
+        def step():
+            zq.ln_quant(X, gamma, beta, 1e-5, Xq=Xq, s_tok=st)
+            fn(Xq, st, Wq, sg, b, Y=Y)
+
+        step()
+        torch.cuda.synchronize()
+        ref = Y.clone()
+        Y.zero_()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(Y, ref)
+        outs[bits] = ref
+    assert zq.device_status()[0] == zq.ZQ_OK

@@ -21,8 +21,7 @@ MUTATIONS = {
     "nibble_shift": ("(uint8_t)(lo | (hi << 4))", "(uint8_t)((lo << 4) | hi)"),
     "ln_mean_sign": ("float d = h2f(x[k]) - mean;", "float d = h2f(x[k]) + mean;"),
     "ln_var_drop_mean": ("double var_d = e2_d - msq;", "double var_d = e2_d;"),
-    "ln_unbiased_var": ("double e2_d = (((double)hi * 0x1p64 + (double)lo) * 0x1p-48) / (double)K;",
-                        "double e2_d = (((double)hi * 0x1p64 + (double)lo) * 0x1p-48) / (double)(K - 1);"),
+    "ln_unbiased_var": ("double c2 = 0x1p-48 / (double)K;", "double c2 = 0x1p-48 / (double)(K - 1);"),
     "gemm_reversed_k": ("for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];",
                         "for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[K - 1 - k];"),
     "dequant_row_scale_swapped": ("v = v * s_grp[zqo_group_of(o, N, g)];\n            v = v + (bias ? h2f(bias[o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM + dequant",

@@ -121,6 +121,32 @@ zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
                        int32_t* acc_dbg, zq_stream_t stream);
 
 /*
+ * zq_gemm_w8a8_noalloc -- zq_gemm_w8a8 for callers that must not let a
+ * library allocate device memory: a serving runtime that owns the whole
+ * device memory pool, a process whose memory budget is fixed up front, or
+ * code that cannot afford the device-wide synchronisation that cudaMalloc /
+ * cudaFree may cause.  It has no counterpart in the paper; it exists only
+ * for such callers.
+ *   Same arguments, results and requirements as zq_gemm_w8a8.  The caller
+ *   still owns and passes every input and output.  The scratch memory of the
+ *   split-K reduction (small token counts) comes from a fixed array of
+ *   8 MiB + 64 KiB in device memory that the library declares statically;
+ *   every GPU that loads the library holds it until the process exits, and
+ *   no call of this function allocates or frees anything.
+ *   Limit: when the planned split-K reduction needs more than that, i.e.
+ *   splits * T * N int32 partial sums above 8 MiB, or more than 16384 tile
+ *   counters, the call returns ZQ_ERR_SHAPE without launching.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls on a device share the one array: calls whose work may overlap
+ *   on the GPU (for example on different streams) race on it and give wrong
+ *   results.  Each call clears the counters it uses, on `stream`.
+ */
+zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
+                               const float* s_grp, int g, const void* bias, int T, int N, int K,
+                               void* Y, int32_t* acc_dbg, zq_stream_t stream);
+
+/*
  * zq_device_status -- synchronize `stream`, then read and clear the status
  * word of the current device.  Returns ZQ_OK, ZQ_ERR_TIMEOUT when a kernel
  * gave up a bounded wait since the last call (*detail receives the kernel's

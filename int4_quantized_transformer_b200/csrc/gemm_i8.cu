@@ -787,3 +787,128 @@ extern "C" zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const ui
                                   int K, void* Y, int32_t* acc_dbg, zq_stream_t stream) {
   return zq::gemm_entry(true, Xq, s_tok, Wq4, s_grp, g, bias, T, N, K, Y, acc_dbg, stream);
 }
+
+// ----------------------------------------------------------------------------
+// Allocation-free variant of zq_gemm_w8a8.
+//
+// The split-K reduction of the weight-streaming tiling needs scratch memory
+// (one int32 partial-sum slice per K split plus per-tile arrival counters).
+// zq_gemm_w8a8 allocates that lazily with cudaMalloc.  Some callers cannot
+// let a library allocate: a serving runtime that owns the whole device
+// memory pool, a process whose memory budget is fixed up front, or code that
+// must never trigger the device-wide synchronisation cudaMalloc/cudaFree can
+// imply.  This variant takes its scratch from a fixed array in device memory
+// that exists from library load until process exit on every GPU that loads
+// the library.
+namespace zq {
+namespace {
+
+constexpr size_t kNoAllocPartialInts = (8u << 20) / sizeof(int32_t);  // 8 MiB of partial sums
+constexpr size_t kNoAllocCounters = 16384;                           // 64 KiB of counters
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocPartialInts + kNoAllocCounters];
+
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_ptr[64] = {};
+
+// Device address of the fixed scratch on the current device.  Host code
+// cannot use the array's name as a device pointer; the address is looked up
+// once per device, with that device current.
+cudaError_t noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace zq
+
+extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
+                                          const float* s_grp, int g, const void* bias, int T,
+                                          int N, int K, void* Y, int32_t* acc_dbg,
+                                          zq_stream_t stream) {
+  using namespace zq;
+  if (T < 0 || N < 8 || N % 8 != 0 || K < 16 || K % 16 != 0 || K > 133136) return ZQ_ERR_SHAPE;
+  if (g < 1 || g > N) return ZQ_ERR_SHAPE;
+  if (T == 0) return ZQ_OK;
+  if (!Xq || !s_tok || !Wq || !s_grp || !Y) return ZQ_ERR_NULL;
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (acc_dbg && !aligned16(acc_dbg)))
+    return ZQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+
+  const int forced_path = option(ZQ_OPT_GEMM_PATH);
+  Plan plan;
+  if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
+    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K));
+  } else {
+    const int fbn = option(ZQ_OPT_GEMM_BN);
+    if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
+    plan = plan_trows(T, N, K, sms, fbn);
+  }
+
+  int* status = device_status_ptr();
+  if (!status) return ZQ_ERR_CUDA;
+
+  GemmParams gp{};
+  gp.s_tok = s_tok;
+  gp.s_grp = s_grp;
+  gp.bias = static_cast<const __half*>(bias);
+  gp.Y = static_cast<__half*>(Y);
+  gp.acc_dbg = acc_dbg;
+  gp.status = status;
+  gp.T = T;
+  gp.N = N;
+  gp.K = K;
+  gp.g = g;
+  gp.m_tiles = plan.m_tiles;
+  gp.n_tiles = plan.n_tiles;
+  gp.k_blocks = plan.k_blocks;
+  gp.splits = plan.splits;
+  gp.kb_per_split = plan.kb_per_split;
+  gp.num_units = plan.units;
+  if (plan.wrows && plan.splits > 1) {
+    const size_t partial = static_cast<size_t>(plan.splits) * T * N;
+    const size_t counters = static_cast<size_t>(plan.m_tiles) * plan.n_tiles * 8;
+    if (partial > kNoAllocPartialInts || counters > kNoAllocCounters) return ZQ_ERR_SHAPE;
+    int32_t* scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return ZQ_ERR_CUDA;
+    // The arrival counters must start at zero; the array keeps whatever the
+    // previous call left there.  The partial sums need no clearing.
+    int* ctr = reinterpret_cast<int*>(scratch + kNoAllocPartialInts);
+    if (cudaMemsetAsync(ctr, 0, counters * sizeof(int), st) != cudaSuccess) return ZQ_ERR_CUDA;
+    gp.ws = scratch;
+    gp.counters = ctr;
+  }
+
+  const int act_rows = plan.wrows ? plan.bn : BM;
+  const int w_rows = plan.wrows ? BM : plan.bn;
+  CUtensorMap ma, mw, my;
+  if (!encode_tma_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, T, K, BK, act_rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return ZQ_ERR_CUDA;
+  if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, BK, w_rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return ZQ_ERR_CUDA;
+  if (!encode_tma_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
+                     32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return ZQ_ERR_CUDA;
+
+  int grid = std::min(plan.units, sms);
+  const int cap = option(ZQ_OPT_MAX_CTAS);
+  if (cap > 0) grid = std::min(grid, cap);
+  const cudaError_t e = plan.wrows ? dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st)
+                                   : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}

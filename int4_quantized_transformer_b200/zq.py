@@ -23,7 +23,7 @@ OPT_GEMM_PATH, OPT_GEMM_BN, OPT_SPLIT_K, OPT_MAX_CTAS = 1, 2, 3, 4
 EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
-    "zq_debug_wait_timeout",
+    "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc",
 )
 
 
@@ -50,6 +50,7 @@ def _load():
         "zq_set_option": ([I, I], I),
         "zq_get_option": ([I], I),
         "zq_debug_wait_timeout": ([P], I),
+        "zq_gemm_w8a8_noalloc": ([P, P, P, P, I, P, I, I, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -190,6 +191,13 @@ def gemm_w4a8(Xq, s_tok, Wq4, s_grp, bias=None, Y=None, acc_dbg=None, stream=Non
     """As gemm_w8a8 with packed INT4 weights uint8 [N, K/2]."""
     return _gemm(_lib.zq_gemm_w4a8, "zq_gemm_w4a8", Xq, s_tok, Wq4, s_grp, bias, Wq4.shape[0], Y,
                  acc_dbg, stream, 4)
+
+
+def gemm_w8a8_noalloc(Xq, s_tok, Wq, s_grp, bias=None, Y=None, acc_dbg=None, stream=None):
+    """gemm_w8a8 without any device allocation by the library: the split-K
+    scratch comes from a fixed array in device memory (zq_gemm_w8a8_noalloc)."""
+    return _gemm(_lib.zq_gemm_w8a8_noalloc, "zq_gemm_w8a8_noalloc", Xq, s_tok, Wq, s_grp, bias,
+                 Wq.shape[0], Y, acc_dbg, stream, 8)
 
 
 def debug_wait_timeout(stream=None):

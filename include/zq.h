@@ -56,7 +56,9 @@ int zq_abi_version(void);
  * quantization (Sec. 3.4 "Group-wise Weight Quantization", Eq. 2).
  *   W      fp16 [N][K]; N rows split into g contiguous groups.
  *   bits   8: Wq is int8 [N][K].  4: Wq is uint8 [N][K/2], two signed
- *          two's-complement nibbles per byte, low nibble = even k.
+ *          two's-complement nibbles per byte: of each eight consecutive k
+ *          (k = 8m..8m+7), byte 4m+i of the row holds k = 8m+i in its low
+ *          nibble and k = 8m+4+i in its high nibble.
  *   s_grp  fp32 [g]: S_i = amax_i / qmax with amax_i = max |W| over group i,
  *          qmax = 127 (bits 8) or 7 (bits 4).  q = clamp(rne(w * (qmax/amax_i)),
  *          -qmax, qmax); a group that is all zero gets S_i = 0 and q = 0.
@@ -114,7 +116,7 @@ zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
  * get INT4": FFN weights in INT4).  Wq4 is uint8 [N][K/2] in the layout of
  * zq_quantize_weights_groupwise(bits=4); the kernel unpacks the nibbles to
  * int8 in shared memory before each tensor-core MMA.
- * Requirements as zq_gemm_w8a8, plus K % 32 == 0.
+ * Requirements as zq_gemm_w8a8, plus K % 32 == 0 and K <= 132096.
  */
 zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
                        const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,

@@ -27,8 +27,9 @@
 //              accumulator is ready ("read the two groups of quantization
 //              scales in advance");
 //   warps 10-13 (W4A8 only) unpack: packed signed INT4 weights, staged by TMA,
-//              are sign-extended to int8 and written into the MMA's
-//              128B-swizzled K-major layout in shared memory.
+//              are widened to int8 (as codes*16, two logic ops per eight
+//              nibbles) and written into the MMA's 128B-swizzled K-major
+//              layout in shared memory; the epilogue divides by 16 exactly.
 //
 // Every wait on an mbarrier is bounded (about a second), after which the
 // kernel records the wait site in the device status word and every role
@@ -145,15 +146,14 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
   return ok != 0;
 }
 
-// Sign-extend the eight nibbles of w (low nibble first) into eight int8.
-__device__ __forceinline__ void unpack8(uint32_t w, uint32_t& o0, uint32_t& o1) {
-  const uint32_t lo = w & 0x0F0F0F0Fu;         // nibbles 0,2,4,6
-  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // nibbles 1,3,5,7
-  uint32_t a = __byte_perm(lo, hi, 0x5140);    // 0,1,2,3
-  uint32_t b = __byte_perm(lo, hi, 0x7362);    // 4,5,6,7
-  // per byte x in [0,15]: ((x ^ 8) + 0x78) ^ 0x80 == x - 16*(x >= 8), no carries
-  o0 = ((a ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-  o1 = ((b ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+// Widen one 32-bit word of packed INT4 codes (eight consecutive k: byte i
+// holds k = i in its low nibble and k = 4 + i in its high nibble) to eight
+// int8 values in k order.  Each nibble lands in the high half of its byte,
+// so the bytes are the codes times 16 (exact two's complement, no carries
+// between bytes); the epilogue divides the int32 accumulator by 16 exactly.
+__device__ __forceinline__ void unpack8_x16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  lo = (w << 4) & 0xF0F0F0F0u;  // k = 0..3
+  hi = w & 0xF0F0F0F0u;         // k = 4..7
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -215,6 +215,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // Set-up above touches no global memory; everything below may read what
+  // the previous kernel of the stream wrote, or overwrite what it reads.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -445,6 +449,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         tmem_ld_32x32b_x32(t_row + c0, a0);
         if (two) tmem_ld_32x32b_x32(t_row + c0 + 32, a1);
         tmem_ld_wait();
+        if (C::W4) {  // INT4 weights were widened as codes*16: exact division
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
+            a1[j] = static_cast<uint32_t>(static_cast<int>(a1[j]) >> 4);
+          }
+        }
         process(a0, c0);
         if (two) process(a1, c0 + 32);
       }
@@ -472,17 +483,32 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           __threadfence();
           const int o = row_idx;
           if (o < p.N) {
-            for (int c = cb; c < ce; ++c) {
-              const int tok = t.n * BN + c;
-              if (tok >= p.T) break;
-              const size_t idx = static_cast<size_t>(tok) * p.N + o;
-              const size_t plane = static_cast<size_t>(p.T) * p.N;
-              int a = 0;
-              for (int sp = 0; sp < p.splits; ++sp) a += __ldcg(p.ws + sp * plane + idx);
-              float v = __fmul_rn(__int2float_rn(a), colv[c]);
-              v = __fadd_rn(__fmul_rn(v, rscale), rbias);
-              p.Y[idx] = __float2half_rn(v);
-              if (p.acc_dbg) p.acc_dbg[idx] = a;
+            const size_t plane = static_cast<size_t>(p.T) * p.N;
+            // eight token columns at a time, so the partial-sum loads of all
+            // splits are independent and in flight together
+            for (int c = cb; c < ce && t.n * BN + c < p.T; c += 8) {
+              int a[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) a[j] = 0;
+              for (int sp = 0; sp < p.splits; ++sp) {
+                const int32_t* src = p.ws + sp * plane + o;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const int tok = t.n * BN + c + j;
+                  if (c + j < ce && tok < p.T) a[j] += __ldcg(src + static_cast<size_t>(tok) * p.N);
+                }
+              }
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int tok = t.n * BN + c + j;
+                if (c + j < ce && tok < p.T) {
+                  const size_t idx = static_cast<size_t>(tok) * p.N + o;
+                  float v = __fmul_rn(__int2float_rn(a[j]), colv[c + j]);
+                  v = __fadd_rn(__fmul_rn(v, rscale), rbias);
+                  p.Y[idx] = __float2half_rn(v);
+                  if (p.acc_dbg) p.acc_dbg[idx] = a[j];
+                }
+              }
             }
           }
         }
@@ -510,8 +536,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             const int r = c >> 3, j = c & 7;
             const uint2 pk = *reinterpret_cast<const uint2*>(src + r * (BK / 2) + j * 8);
             uint4 o;
-            unpack8(pk.x, o.x, o.y);
-            unpack8(pk.y, o.z, o.w);
+            unpack8_x16(pk.x, o.x, o.y);
+            unpack8_x16(pk.y, o.z, o.w);
             *reinterpret_cast<uint4*>(dst + r * BK + ((j ^ (r & 7)) << 4)) = o;
           }
           fence_proxy_async_smem();
@@ -658,7 +684,9 @@ cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUten
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  gemm_i8_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mw, my, gp);
+  cudaError_t e = launch_pdl(gemm_i8_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
+                             static_cast<size_t>(C::SMEM_BYTES), st, ma, mw, my, gp);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -686,7 +714,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
                      const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,
                      int32_t* acc_dbg, zq_stream_t stream) {
   if (T < 0 || N < 8 || N % 8 != 0 || K < 16 || K % 16 != 0 || K > 133136) return ZQ_ERR_SHAPE;
-  if (w4 && K % 32 != 0) return ZQ_ERR_SHAPE;
+  if (w4 && (K % 32 != 0 || K > 132096)) return ZQ_ERR_SHAPE;
   if (g < 1 || g > N) return ZQ_ERR_SHAPE;
   if (T == 0) return ZQ_OK;
   if (!Xq || !s_tok || !Wq || !s_grp || !Y) return ZQ_ERR_NULL;

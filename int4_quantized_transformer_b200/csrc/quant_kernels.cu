@@ -9,7 +9,8 @@
 //    the int8 row and its scale are written back.
 //  * wquant: group-wise weight quantization ("Group-wise Weight
 //    Quantization", Eq. 2), one CTA per group of contiguous output rows,
-//    with optional packing of two signed INT4 codes per byte.
+//    with optional packing of two signed INT4 codes per byte (of each eight
+//    consecutive k, byte i holds k = i and k = 4 + i).
 //
 // Every floating-point step uses an explicit round-to-nearest intrinsic so
 // that the compiler cannot contract it into an FMA: results are bit-exact
@@ -17,6 +18,7 @@
 #include <cuda_fp16.h>
 
 #include "zq_internal.h"
+#include "zq_ptx.cuh"
 
 namespace zq {
 namespace {
@@ -39,6 +41,14 @@ __device__ __forceinline__ uint32_t quant_code(float y, float inv, float qmax) {
   return rne_low_byte(v);
 }
 
+// Token quantization of one element: as quant_code with qmax = 127, without
+// the clamp, which cannot bind here: amax = max|y| over the row and
+// inv = fp32(127/amax), so |y*inv| <= 127*(1+2^-24)^2 and its rounding to the
+// nearest integer is at most 127.
+__device__ __forceinline__ uint32_t token_code(float y, float inv) {
+  return rne_low_byte(__fmul_rn(y, inv));
+}
+
 __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   uint32_t lo = __byte_perm(a, b, 0x0040);
   uint32_t hi = __byte_perm(c, d, 0x0040);
@@ -48,35 +58,39 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 // --------------------------------------------------------------- ln_quant
 
 struct RowSums {
-  long long s1;                // sum of a = x * 2^24 (an integer for every finite fp16 x)
-  unsigned long long p, q, r;  // sum of a^2 = p*2^40 + q*2^21 + r, with |a| = ah*2^20 + al
+  long long s1;            // sum of a = x * 2^24 (an integer for every finite fp16 x)
+  unsigned long long p;    // sum of ah^2    } with a = ah*2^20 + al, ah = floor(x*16),
+  long long q;             // sum of ah*al   } al in [0, 2^20): a^2 = p*2^40 + q*2^21 + r
+  unsigned long long r;    // sum of al^2    }
 };
 
-// Per-thread partial sums, kept in 32-bit where that is exact: a thread adds
-// at most 32 elements, so sum(+-ah) and sum(+-al) stay below 2^26.
+// Per-thread partial sums: a thread adds at most 32 elements, so sum(ah) and
+// sum(al) stay below 2^26 in magnitude and fit 32-bit integers.
 struct ThreadSums {
   int s1h, s1l;
-  unsigned long long p, q, r;
+  unsigned long long p, r;
+  long long q;
 };
 
 // Adds one fp16 value x (already converted to fp32, exactly) to the exact
-// sums.  |a| = |x|*2^24 = ah*2^20 + al with ah = floor(|x|*16) and
-// al = frac(|x|*16)*2^20, both below 2^20.  The integer and fractional parts
-// come from the fp32 "magic number" technique: adding 2^23 with rounding
-// toward zero leaves floor(v) in the low mantissa bits of the sum (v < 2^20),
-// and the remaining fraction is an exact multiple of 2^-20.
+// sums.  a = x*2^24 = ah*2^20 + al with ah = floor(x*16) (|ah| <= 2^20) and
+// al = (x*16 - ah)*2^20 in [0, 2^20).  Both come from the fp32 "magic
+// number" technique: adding 1.5*2^23 with rounding toward zero leaves
+// floor(v) in the low mantissa bits (|v| < 2^20, the sum stays in
+// [2^23, 2^24) where the spacing is 1), and the remaining fraction is an
+// exact multiple of 2^-20.
 __device__ __forceinline__ void add_exact(ThreadSums& s, float x) {
-  const float v = __fmul_rn(fabsf(x), 16.0f);               // |x|*16 < 2^20, exact
-  const float t = __fadd_rz(v, 8388608.0f);                 // 2^23 + floor(v)
-  const uint32_t ah = __float_as_uint(t) - 0x4B000000u;
-  const float fr = __fsub_rn(v, __fsub_rn(t, 8388608.0f));  // v - floor(v), exact
-  const uint32_t al = __float_as_uint(__fmaf_rn(fr, 1048576.0f, 8388608.0f)) - 0x4B000000u;
-  const int sg = (__float_as_int(x) >> 31) | 1;             // -1 or +1
-  s.s1h += sg * static_cast<int>(ah);
-  s.s1l += sg * static_cast<int>(al);
-  s.p += static_cast<unsigned long long>(ah) * ah;
-  s.q += static_cast<unsigned long long>(ah) * al;
-  s.r += static_cast<unsigned long long>(al) * al;
+  const float v = __fmul_rn(x, 16.0f);                       // exact, |v| < 2^20
+  const float t = __fadd_rz(v, 12582912.0f);                 // 1.5*2^23 + floor(v)
+  const int ah = static_cast<int>(__float_as_uint(t) - 0x4B400000u);
+  const float fr = __fsub_rn(v, __fsub_rn(t, 12582912.0f));  // v - floor(v), exact
+  const int al = static_cast<int>(__float_as_uint(__fmaf_rn(fr, 1048576.0f, 8388608.0f)) -
+                                  0x4B000000u);
+  s.s1h += ah;
+  s.s1l += al;
+  s.p += static_cast<unsigned long long>(static_cast<long long>(ah) * ah);
+  s.q += static_cast<long long>(ah) * al;
+  s.r += static_cast<unsigned long long>(al) * static_cast<unsigned int>(al);
 }
 
 __device__ __forceinline__ void warp_sum(RowSums& s) {
@@ -101,9 +115,9 @@ __device__ __forceinline__ float warp_max(float v) {
 // rstd = 1/sqrt(fp32(var) + eps) in fp32.
 __device__ __forceinline__ void row_stats(const RowSums& s, double c1, double c2, float eps,
                                           float& mean, float& rstd) {
-  const unsigned __int128 s2 = (static_cast<unsigned __int128>(s.p) << 40) +
-                               (static_cast<unsigned __int128>(s.q) << 21) +
-                               static_cast<unsigned __int128>(s.r);
+  const __int128 s2s = (static_cast<__int128>(s.p) << 40) + (static_cast<__int128>(s.q) << 21) +
+                       static_cast<__int128>(s.r);
+  const unsigned __int128 s2 = static_cast<unsigned __int128>(s2s);  // a sum of squares: >= 0
   const unsigned long long hi = static_cast<unsigned long long>(s2 >> 64);
   const unsigned long long lo = static_cast<unsigned long long>(s2);
   const double mean_d = __dmul_rn(__ll2double_rn(s.s1), c1);
@@ -137,6 +151,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
   const int lane = threadIdx.x & 31;
   const int nvec = K / 8;
   const bool ln = gamma != nullptr;
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   const int rows_per_iter = gridDim.x * RPB;
   const int iters = (T + rows_per_iter - 1) / rows_per_iter;
@@ -241,8 +257,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __half22float2(h[e]);
-            c[2 * e] = quant_code(f.x, inv, 127.0f);
-            c[2 * e + 1] = quant_code(f.y, inv, 127.0f);
+            c[2 * e] = token_code(f.x, inv);
+            c[2 * e + 1] = token_code(f.y, inv);
           }
           uint2 out;
           out.x = pack4(c[0], c[1], c[2], c[3]);
@@ -270,7 +286,9 @@ cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, int T, 
   if (grid > need) grid = need;
   const double c1 = 0x1p-24 / static_cast<double>(K);
   const double c2 = 0x1p-48 / static_cast<double>(K);
-  ln_quant_kernel<W, VPT><<<grid, threads, 0, st>>>(X, g, b, T, K, eps, c1, c2, Xq, s, Y);
+  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, T, K, eps,
+                 c1, c2, Xq, s, Y);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -303,6 +321,8 @@ __global__ void __launch_bounds__(512) wquant_kernel(const __half* __restrict__ 
                                                      int g, int bits, void* __restrict__ Wq,
                                                      float* __restrict__ s_grp) {
   __shared__ float red[16];
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int i = blockIdx.x;
   const long long r0 = (static_cast<long long>(i) * N + g - 1) / g;
   const long long r1 = (static_cast<long long>(i + 1) * N + g - 1) / g;
@@ -333,10 +353,11 @@ __global__ void __launch_bounds__(512) wquant_kernel(const __half* __restrict__ 
       out.y = pack4(c[4], c[5], c[6], c[7]);
       reinterpret_cast<uint2*>(static_cast<int8_t*>(Wq) + r0 * K)[v] = out;
     } else {
-      // two's-complement nibbles, low nibble = even k
+      // two's-complement nibbles; of eight consecutive k, byte i holds
+      // k = i (low nibble) and k = 4 + i (high nibble)
       uint32_t out = 0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) out |= (c[e] & 0xFu) << (4 * e);
+      for (int e = 0; e < 4; ++e) out |= ((c[e] & 0xFu) | ((c[e + 4] & 0xFu) << 4)) << (8 * e);
       reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(Wq) + r0 * (K / 2))[v] = out;
     }
   }
@@ -386,6 +407,8 @@ extern "C" zq_status zq_quantize_weights_groupwise(const void* W, int N, int K, 
   if (!W || !Wq || !s_grp) return ZQ_ERR_NULL;
   if (!aligned16(W) || !aligned16(Wq)) return ZQ_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  wquant_kernel<<<g, 512, 0, st>>>(static_cast<const __half*>(W), N, K, g, bits, Wq, s_grp);
+  if (launch_pdl(wquant_kernel, dim3(g), dim3(512), 0, st, static_cast<const __half*>(W), N, K, g,
+                 bits, Wq, s_grp) != cudaSuccess)
+    return ZQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }

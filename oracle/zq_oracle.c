@@ -31,7 +31,8 @@
  *   R5 Scales are fp32.
  *   R6 group(o) = floor(o*g/N): g contiguous groups even when g does not
  *      divide N.
- *   R7 INT4: two's-complement nibbles, two per byte, low nibble = even k.
+ *   R7 INT4: two's-complement nibbles, two per byte; of each eight
+ *      consecutive k, byte i holds k = i (low nibble) and k = 4 + i (high).
  *   R8 "round" = round half to even.
  *   R9 Epilogue: y = fp16( ((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]) ),
  *      each a separate IEEE round-to-nearest op (no contraction).
@@ -125,28 +126,34 @@ int zqo_quantize_weights_groupwise(const uint16_t *W, int N, int K, int g, int b
     return 0;
 }
 
-/* R7: byte j of row o = (q[o,2j] & 0xF) | ((q[o,2j+1] & 0xF) << 4).  K even. */
+/* R7: INT4 codes, two per byte.  Row o is cut into blocks of eight
+ * consecutive k; block m is stored in bytes 4m..4m+3 of the row, and byte
+ * 4m+i holds q[o, 8m+i] in its low nibble and q[o, 8m+4+i] in its high
+ * nibble (two's complement).  K must be a multiple of 8. */
 int zqo_pack_int4(const int8_t *q, int N, int K, uint8_t *packed) {
-    if (K % 2) return -1;
+    if (K % 8) return -1;
     for (int o = 0; o < N; ++o)
-        for (int j = 0; j < K / 2; ++j) {
-            unsigned lo = (unsigned)q[(size_t)o * K + 2 * j] & 0xFu;
-            unsigned hi = (unsigned)q[(size_t)o * K + 2 * j + 1] & 0xFu;
-            packed[(size_t)o * (K / 2) + j] = (uint8_t)(lo | (hi << 4));
-        }
+        for (int m = 0; m < K / 8; ++m)
+            for (int i = 0; i < 4; ++i) {
+                unsigned lo = (unsigned)q[(size_t)o * K + 8 * m + i] & 0xFu;
+                unsigned hi = (unsigned)q[(size_t)o * K + 8 * m + 4 + i] & 0xFu;
+                packed[(size_t)o * (K / 2) + 4 * m + i] = (uint8_t)(lo | (hi << 4));
+            }
     return 0;
 }
 
+static int sext4(unsigned v) { return v >= 8 ? (int)v - 16 : (int)v; }
+
 /* Inverse of zqo_pack_int4: sign-extend each nibble. */
 int zqo_unpack_int4(const uint8_t *packed, int N, int K, int8_t *q) {
-    if (K % 2) return -1;
+    if (K % 8) return -1;
     for (int o = 0; o < N; ++o)
-        for (int j = 0; j < K / 2; ++j) {
-            unsigned b = packed[(size_t)o * (K / 2) + j];
-            int lo = (int)(b & 0xFu), hi = (int)(b >> 4);
-            q[(size_t)o * K + 2 * j] = (int8_t)(lo >= 8 ? lo - 16 : lo);
-            q[(size_t)o * K + 2 * j + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
-        }
+        for (int m = 0; m < K / 8; ++m)
+            for (int i = 0; i < 4; ++i) {
+                unsigned b = packed[(size_t)o * (K / 2) + 4 * m + i];
+                q[(size_t)o * K + 8 * m + i] = (int8_t)sext4(b & 0xFu);
+                q[(size_t)o * K + 8 * m + 4 + i] = (int8_t)sext4(b >> 4);
+            }
     return 0;
 }
 

@@ -121,8 +121,9 @@ def quantize_weights_groupwise(W, g: int, bits: int):
 
 
 def pack_int4(q):
-    """Two signed INT4 weights per byte, low nibble = even k (reading of the
-    paper's W4 storage, Sec. 3.4 "Which weights get INT4")."""
+    """Two signed INT4 weights per byte: of each eight consecutive k, byte i
+    holds k = i in its low nibble and k = 4 + i in its high nibble (reading of
+    the paper's W4 storage, Sec. 3.4 "Which weights get INT4")."""
     q = np.ascontiguousarray(q, dtype=np.int8)
     N, K = q.shape
     out = np.empty((N, K // 2), np.uint8)

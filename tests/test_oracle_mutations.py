@@ -18,7 +18,8 @@ MUTATIONS = {
     "ties_away": ("return nearbyintf(v);", "return roundf(v);"),
     "scale_qmax_plus_one": ("return amax / (float)qmax;", "return amax / (float)(qmax + 1);"),
     "group_ceil": ("return (int)(((int64_t)o * g) / N);", "return (int)(((int64_t)o * g + N - 1) / N);"),
-    "nibble_shift": ("(uint8_t)(lo | (hi << 4))", "(uint8_t)((lo << 4) | hi)"),
+    "nibble_swap": ("packed[(size_t)o * (K / 2) + 4 * m + i] = (uint8_t)(lo | (hi << 4));",
+                    "packed[(size_t)o * (K / 2) + 4 * m + i] = (uint8_t)(hi | (lo << 4));"),
     "ln_mean_sign": ("float d = h2f(x[k]) - mean;", "float d = h2f(x[k]) + mean;"),
     "ln_var_drop_mean": ("double var_d = e2_d - msq;", "double var_d = e2_d;"),
     "ln_unbiased_var": ("double c2 = 0x1p-48 / (double)K;", "double c2 = 0x1p-48 / (double)(K - 1);"),

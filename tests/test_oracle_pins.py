@@ -123,17 +123,20 @@ def test_int4_pack_golden_and_round_trip():
         for line in f:
             line = line.split("#")[0].strip()
             if line:
-                a, b, byte = line.split()
-                rows.append((int(a), int(b), int(byte, 16)))
-    q = np.array([[a, b] for a, b, _ in rows], np.int8).reshape(1, -1)
+                q, b = line.split("->")
+                rows.append(([int(v) for v in q.split()], [int(v, 16) for v in b.split()]))
+    q = np.array([r[0] for r in rows], np.int8).reshape(1, -1)
     packed = oracle.pack_int4(q)
-    assert packed.tolist()[0] == [byte for _, _, byte in rows]
-    # every nibble pair survives pack -> unpack
+    assert packed.tolist()[0] == [byte for r in rows for byte in r[1]]
+    # every nibble pair survives pack -> unpack, in both nibble positions
     vals = np.arange(-8, 8)
-    pairs = np.array(np.meshgrid(vals, vals)).reshape(2, -1).T.reshape(1, -1).astype(np.int8)
-    p = oracle.pack_int4(pairs)
-    assert p.nbytes == pairs.size // 2
-    assert np.array_equal(oracle.unpack_int4(p, pairs.shape[1]), pairs)
+    pairs = np.array(np.meshgrid(vals, vals)).reshape(2, -1).T  # 256 (lo, hi) pairs
+    q = np.zeros((1, 256 * 8), np.int8)
+    q[0, 0::8], q[0, 4::8] = pairs[:, 0], pairs[:, 1]
+    q[0, 3::8], q[0, 7::8] = pairs[:, 1], pairs[:, 0]
+    p = oracle.pack_int4(q)
+    assert p.nbytes == q.size // 2
+    assert np.array_equal(oracle.unpack_int4(p, q.shape[1]), q)
 
 
 # ------------------------------------------------------------------- LayerNorm

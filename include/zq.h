@@ -77,9 +77,11 @@ zq_status zq_quantize_weights_groupwise(const void* W, int N, int K, int g, int 
  *   beta   fp16 [K] or NULL (= 0).  Ignored when gamma is NULL.
  *   eps    LayerNorm epsilon (added to the biased variance).
  *   Xq     int8 [T][K] output, s_tok fp32 [T] output:
- *          y = fp16(((x - mean) * rstd) * gamma + beta), mean and biased
- *          variance computed exactly (integer sums of x*2^24 and its square),
- *          rstd = fp32(1/sqrt(var + eps)) in fp64;
+ *          y = fp16(((x - mean) * rstd) * gamma + beta) in fp32, with
+ *          mean = S/K and biased var = Q/K, where S sums x and Q sums
+ *          (x - mean)^2 in a fixed order: chunks of 8 consecutive values in
+ *          index order, chunk sums combined by a zero-padded pairwise tree;
+ *          rstd = 1/sqrt(var + eps);
  *          s_tok[t] = amax_t/127 with amax_t = max_k |y|,
  *          Xq = clamp(rne(y * (127/amax_t)), -127, 127); zero rows give 0.
  *   Y_ln   fp16 [T][K] or NULL: also store y (unfused form, for checking).

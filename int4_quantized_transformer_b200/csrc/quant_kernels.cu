@@ -3,8 +3,9 @@
 //
 //  * ln_quant: fused LayerNorm + token-wise dynamic INT8 quantization
 //    ("Kernel fusion for token-wise activation quantization", Fig. 2 right):
-//    each row is read once into registers with 128-bit loads, its exact
-//    statistics, fp16 LayerNorm output and absmax are reduced with warp
+//    each row is read once into registers with 128-bit loads; its mean and
+//    variance (fp32 sums in a fixed chunk-and-tree order, two passes over
+//    the registers), fp16 LayerNorm output and absmax are reduced with warp
 //    shuffles (plus shared memory when several warps share a row), and only
 //    the int8 row and its scale are written back.
 //  * wquant: group-wise weight quantization ("Group-wise Weight
@@ -57,77 +58,60 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 
 // --------------------------------------------------------------- ln_quant
 
-struct RowSums {
-  long long s1;            // sum of a = x * 2^24 (an integer for every finite fp16 x)
-  unsigned long long p;    // sum of ah^2    } with a = ah*2^20 + al, ah = floor(x*16),
-  long long q;             // sum of ah*al   } al in [0, 2^20): a^2 = p*2^40 + q*2^21 + r
-  unsigned long long r;    // sum of al^2    }
-};
-
-// Per-thread partial sums: a thread adds at most 32 elements, so sum(ah) and
-// sum(al) stay below 2^26 in magnitude and fit 32-bit integers.
-struct ThreadSums {
-  int s1h, s1l;
-  unsigned long long p, r;
-  long long q;
-};
-
-// Adds one fp16 value x (already converted to fp32, exactly) to the exact
-// sums.  a = x*2^24 = ah*2^20 + al with ah = floor(x*16) (|ah| <= 2^20) and
-// al = (x*16 - ah)*2^20 in [0, 2^20).  Both come from the fp32 "magic
-// number" technique: adding 1.5*2^23 with rounding toward zero leaves
-// floor(v) in the low mantissa bits (|v| < 2^20, the sum stays in
-// [2^23, 2^24) where the spacing is 1), and the remaining fraction is an
-// exact multiple of 2^-20.
-__device__ __forceinline__ void add_exact(ThreadSums& s, float x) {
-  const float v = __fmul_rn(x, 16.0f);                       // exact, |v| < 2^20
-  const float t = __fadd_rz(v, 12582912.0f);                 // 1.5*2^23 + floor(v)
-  const int ah = static_cast<int>(__float_as_uint(t) - 0x4B400000u);
-  const float fr = __fsub_rn(v, __fsub_rn(t, 12582912.0f));  // v - floor(v), exact
-  const int al = static_cast<int>(__float_as_uint(__fmaf_rn(fr, 1048576.0f, 8388608.0f)) -
-                                  0x4B000000u);
-  s.s1h += ah;
-  s.s1l += al;
-  s.p += static_cast<unsigned long long>(static_cast<long long>(ah) * ah);
-  s.q += static_cast<long long>(ah) * al;
-  s.r += static_cast<unsigned long long>(al) * static_cast<unsigned int>(al);
-}
-
-__device__ __forceinline__ void warp_sum(RowSums& s) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    s.s1 += __shfl_xor_sync(0xffffffffu, s.s1, o);
-    s.p += __shfl_xor_sync(0xffffffffu, s.p, o);
-    s.q += __shfl_xor_sync(0xffffffffu, s.q, o);
-    s.r += __shfl_xor_sync(0xffffffffu, s.r, o);
-  }
-}
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 
-// mean and rstd from the exact sums, c1 = 2^-24/K and c2 = 2^-48/K (fp64,
-// computed on the host): mean = S1*c1, E[x^2] = S2*c2 with S2 taken to
-// fp64 as hi*2^64 + lo, var = max(E[x^2] - mean^2, 0) (biased) in fp64, then
-// rstd = 1/sqrt(fp32(var) + eps) in fp32.
-__device__ __forceinline__ void row_stats(const RowSums& s, double c1, double c2, float eps,
-                                          float& mean, float& rstd) {
-  const __int128 s2s = (static_cast<__int128>(s.p) << 40) + (static_cast<__int128>(s.q) << 21) +
-                       static_cast<__int128>(s.r);
-  const unsigned __int128 s2 = static_cast<unsigned __int128>(s2s);  // a sum of squares: >= 0
-  const unsigned long long hi = static_cast<unsigned long long>(s2 >> 64);
-  const unsigned long long lo = static_cast<unsigned long long>(s2);
-  const double mean_d = __dmul_rn(__ll2double_rn(s.s1), c1);
-  const double e2 =
-      __dmul_rn(__dadd_rn(__dmul_rn(__ull2double_rn(hi), 0x1p64), __ull2double_rn(lo)), c2);
-  double var = __dsub_rn(e2, __dmul_rn(mean_d, mean_d));
-  if (var < 0.0) var = 0.0;
-  const float r = __fsqrt_rn(__fadd_rn(__double2float_rn(var), eps));
-  rstd = __fdiv_rn(1.0f, r);
-  mean = __double2float_rn(mean_d);
+// Row sums in a fixed order that does not depend on the launch shape.  The
+// row is cut into chunks of eight consecutive elements, each summed in
+// order; the chunk sums, padded with zeros to a power of two, are combined
+// by a pairwise tree (level l adds chunk c + 2^l into chunk c, for c a
+// multiple of 2^(l+1)).  Chunk c sits in thread (c mod RT) of the row, slot
+// c / RT, i.e. lane c mod 32 and "block" b = c / 32 = warp + W*slot, so
+// levels 0..4 are xor-shuffles inside a warp (IEEE addition is commutative,
+// so both partners hold the same bits) and the higher levels are the same
+// tree over the blocks b.  `cs` holds this thread's chunk sums; the result
+// reaches every thread of the row.
+template <int W, int VPT>
+__device__ __forceinline__ float row_tree_sum(float (&cs)[VPT], float* red, int lane, int wrow) {
+  constexpr int VPTP = VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4);  // slots padded to a power of two
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) cs[i] = __fadd_rn(cs[i], __shfl_xor_sync(0xffffffffu, cs[i], o));
+  if (W == 1) {  // blocks are the slots of this thread
+    float b[VPTP];
+#pragma unroll
+    for (int i = 0; i < VPTP; ++i) b[i] = i < VPT ? cs[i] : 0.0f;
+#pragma unroll
+    for (int st = 1; st < VPTP; st <<= 1)
+#pragma unroll
+      for (int i = 0; i < VPTP; i += 2 * st) b[i] = __fadd_rn(b[i], b[i + st]);
+    return b[0];
+  }
+  // W > 1: block b = warp + W*slot; every warp reduces all blocks from
+  // shared memory (lane + 32r = b), first across lanes, then across r.
+  constexpr int NB = W * VPTP;
+  constexpr int NR = NB <= 32 ? 1 : NB / 32;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < VPTP; ++i) red[wrow + W * i] = i < VPT ? cs[i] : 0.0f;
+  }
+  __syncthreads();
+  float v[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) v[r] = (lane + 32 * r < NB) ? red[lane + 32 * r] : 0.0f;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int r = 0; r < NR; ++r) v[r] = __fadd_rn(v[r], __shfl_xor_sync(0xffffffffu, v[r], o));
+#pragma unroll
+  for (int st = 1; st < NR; st <<= 1)
+#pragma unroll
+    for (int r = 0; r < NR; r += 2 * st) v[r] = __fadd_rn(v[r], v[r + st]);
+  return v[0];
 }
 
 // W warps per row, VPT 16-byte vectors (8 halves) per thread.  Blocks hold
@@ -137,12 +121,14 @@ __device__ __forceinline__ void row_stats(const RowSums& s, double c1, double c2
 template <int W, int VPT>
 __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 32) : 8) / 2)
     ln_quant_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
-                    const __half* __restrict__ beta, int T, int K, float eps, double c1,
-                    double c2, int8_t* __restrict__ Xq, float* __restrict__ s_tok,
+                    const __half* __restrict__ beta, int T, int K, float eps,
+                    int8_t* __restrict__ Xq, float* __restrict__ s_tok,
                     __half* __restrict__ Y_ln) {
   constexpr int RT = 32 * W;                // threads per row
   constexpr int RPB = W >= 8 ? 1 : 8 / W;   // rows per block
-  __shared__ RowSums red_s[RPB][W];
+  constexpr int NBLK = W * (VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4));
+  __shared__ float red1[RPB][NBLK];  // block sums of x (W > 1)
+  __shared__ float red2[RPB][NBLK];  // block sums of (x - mean)^2 (W > 1)
   __shared__ float red_m[RPB][W];
 
   const int slot = threadIdx.x / RT;
@@ -170,41 +156,43 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
     }
 
     if (ln) {
-      ThreadSums ts = {0, 0, 0, 0, 0};
+      // mean: chunk sums of x in order, then the pairwise tree
+      float cs[VPT];
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
+        const float2 f0 = __half22float2(h[0]);
+        float acc = __fadd_rn(f0.x, f0.y);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 1; e < 4; ++e) {
           const float2 f = __half22float2(h[e]);
-          add_exact(ts, f.x);
-          add_exact(ts, f.y);
+          acc = __fadd_rn(__fadd_rn(acc, f.x), f.y);
         }
+        cs[i] = acc;  // zero for chunks past the row (x4 is zero there)
       }
-      RowSums s;
-      s.s1 = static_cast<long long>(ts.s1h) * 1048576 + ts.s1l;
-      s.p = ts.p;
-      s.q = ts.q;
-      s.r = ts.r;
-      warp_sum(s);
-      if (W > 1) {
-        if (lane == 0) red_s[slot][warp_in_row] = s;
-        __syncthreads();
-        s = red_s[slot][0];
+      const float mean = __fdiv_rn(row_tree_sum<W, VPT>(cs, red1[slot], lane, warp_in_row),
+                                   static_cast<float>(K));
+      // biased variance: chunk sums of (x - mean)^2 (first square, then
+      // fused multiply-adds), then the same tree
 #pragma unroll
-        for (int w = 1; w < W; ++w) {
-          RowSums t = red_s[slot][w];
-          s.s1 += t.s1;
-          s.p += t.p;
-          s.q += t.q;
-          s.r += t.r;
+      for (int i = 0; i < VPT; ++i) {
+        const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
+        const float2 f0 = __half22float2(h[0]);
+        const float d0 = __fsub_rn(f0.x, mean);
+        const float d1 = __fsub_rn(f0.y, mean);
+        float acc = __fmaf_rn(d1, d1, __fmul_rn(d0, d0));
+#pragma unroll
+        for (int e = 1; e < 4; ++e) {
+          const float2 f = __half22float2(h[e]);
+          const float da = __fsub_rn(f.x, mean);
+          const float db = __fsub_rn(f.y, mean);
+          acc = __fmaf_rn(db, db, __fmaf_rn(da, da, acc));
         }
+        cs[i] = (j + i * RT < nvec) ? acc : 0.0f;  // padding chunks are zero
       }
-      // One lane does the fp64 row arithmetic; the warp gets it by shuffle.
-      float mean = 0.0f, rstd = 0.0f;
-      if (lane == 0) row_stats(s, c1, c2, eps, mean, rstd);
-      mean = __shfl_sync(0xffffffffu, mean, 0);
-      rstd = __shfl_sync(0xffffffffu, rstd, 0);
+      const float var = __fdiv_rn(row_tree_sum<W, VPT>(cs, red2[slot], lane, warp_in_row),
+                                  static_cast<float>(K));
+      const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         const int v = j + i * RT;
@@ -242,7 +230,7 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
       __syncthreads();
 #pragma unroll
       for (int w = 0; w < W; ++w) amax = fmaxf(amax, red_m[slot][w]);
-      __syncthreads();  // red_s / red_m are reused by the next row
+      __syncthreads();  // red1 / red2 / red_m are reused by the next row
     }
     const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
     if (valid) {
@@ -284,10 +272,8 @@ cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, int T, 
   int need = (T + RPB - 1) / RPB;
   int grid = num_sms() * per_sm;
   if (grid > need) grid = need;
-  const double c1 = 0x1p-24 / static_cast<double>(K);
-  const double c2 = 0x1p-48 / static_cast<double>(K);
   e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, T, K, eps,
-                 c1, c2, Xq, s, Y);
+                 Xq, s, Y);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -22,10 +22,11 @@
  *      fp32 multiply per element.
  *   R2 Clamp to [-qmax, qmax] (qmax = 127 or 7): symmetric, and the absmax
  *      scale never produces -128/-8 anyway.
- *   R3 LayerNorm statistics are computed exactly (integer sums of x*2^24 and
- *      of its square), so they do not depend on summation order; mean and
- *      variance are then formed in fp64 and 1/sqrt(var + eps) in fp32
- *      (see zqo_ln_row_stats for the exact sequence of roundings).
+ *   R3 LayerNorm statistics are fp32 sums in a fixed order that does not
+ *      depend on how a kernel splits the row: chunks of 8 consecutive values
+ *      summed in order, chunk sums combined by a zero-padded pairwise tree;
+ *      the variance is the biased two-pass sum of (x - mean)^2
+ *      (see zqo_ln_row_stats).
  *   R4 The fused kernel quantizes its fp16 LayerNorm output (Fig. 2: fused and
  *      unfused compute the same output).
  *   R5 Scales are fp32.
@@ -159,46 +160,64 @@ int zqo_unpack_int4(const uint8_t *packed, int N, int K, int8_t *q) {
 
 /* -------------------------------------------- LayerNorm (reading R3) */
 
-/* Exact row statistics: a_k = x_k * 2^24 is an integer (|a_k| < 2^40) for
- * every finite fp16 x_k.  S1 = sum a_k (int64), S2 = sum a_k^2 (128-bit,
- * returned as two 64-bit halves). */
-void zqo_ln_exact_sums(const uint16_t *x, int K, int64_t *S1, uint64_t *S2_hi, uint64_t *S2_lo) {
-    int64_t s1 = 0;
-    unsigned __int128 s2 = 0;
-    for (int k = 0; k < K; ++k) {
-        int64_t a = (int64_t)((double)h2f(x[k]) * 16777216.0); /* exact */
-        s1 += a;
-        unsigned __int128 m = (unsigned __int128)(a < 0 ? -a : a);
-        s2 += m * m;
-    }
-    *S1 = s1;
-    *S2_hi = (uint64_t)(s2 >> 64);
-    *S2_lo = (uint64_t)s2;
+/* Pairwise tree over n values (n a power of two): level l adds v[c + 2^l]
+ * into v[c] for every c that is a multiple of 2^(l+1).  Returns v[0]. */
+static float tree_sum(float *v, int n) {
+    for (int step = 1; step < n; step *= 2)
+        for (int c = 0; c < n; c += 2 * step) v[c] = v[c] + v[c + step];
+    return v[0];
 }
 
-/* mean and rstd of one row, from the exact sums (biased variance, /K):
- *   c1 = 2^-24/K, c2 = 2^-48/K                      (fp64 divisions)
- *   mean_d = S1*c1, E2 = (hi*2^64 + lo)*c2           (fp64)
- *   var_d  = max(E2 - mean_d^2, 0)                   (fp64)
- *   rstd   = 1/sqrt(fp32(var_d) + eps)               (fp32), mean = fp32(mean_d). */
+static int pow2_at_least(int n) {
+    int p = 1;
+    while (p < n) p *= 2;
+    return p;
+}
+
+/* Row sum in the fixed order of reading R3: the row is cut into chunks of
+ * eight consecutive values (the last one shorter when K is not a multiple of
+ * 8), each chunk summed in index order, and the chunk sums, padded with
+ * zeros to a power of two, combined by the pairwise tree.  With sq != 0 the
+ * summands are (x - mean)^2: the first one squared, the rest accumulated with
+ * fused multiply-adds. */
+static float chunk_tree_sum(const uint16_t *x, int K, int sq, float mean) {
+    int nchunk = (K + 7) / 8;
+    int P = pow2_at_least(nchunk);
+    float *cs = (float *)calloc((size_t)P, sizeof(float));
+    for (int c = 0; c < nchunk; ++c) {
+        int k0 = 8 * c, k1 = k0 + 8 < K ? k0 + 8 : K;
+        float acc;
+        if (sq) {
+            float d = h2f(x[k0]) - mean;
+            acc = d * d;
+            for (int k = k0 + 1; k < k1; ++k) {
+                d = h2f(x[k]) - mean;
+                acc = fmaf(d, d, acc);
+            }
+        } else {
+            acc = h2f(x[k0]);
+            for (int k = k0 + 1; k < k1; ++k) acc = acc + h2f(x[k]);
+        }
+        cs[c] = acc;
+    }
+    float r = tree_sum(cs, P);
+    free(cs);
+    return r;
+}
+
+/* mean and rstd of one row (reading R3, all fp32, biased variance):
+ *   mean = S/K with S the fixed-order sum of x,
+ *   var  = Q/K with Q the fixed-order sum of (x - mean)^2 (two passes),
+ *   rstd = 1/sqrt(var + eps). */
 void zqo_ln_row_stats(const uint16_t *x, int K, float eps, float *mean_out, float *rstd_out,
                       double *mean_d_out, double *var_d_out) {
-    int64_t S1;
-    uint64_t hi, lo;
-    zqo_ln_exact_sums(x, K, &S1, &hi, &lo);
-    double c1 = 0x1p-24 / (double)K;
-    double c2 = 0x1p-48 / (double)K;
-    double mean_d = (double)S1 * c1;
-    double e2_d = ((double)hi * 0x1p64 + (double)lo) * c2;
-    double msq = mean_d * mean_d;
-    double var_d = e2_d - msq;
-    if (var_d < 0.0) var_d = 0.0;
-    float vf = (float)var_d;
-    float r = sqrtf(vf + eps);
+    float mean = chunk_tree_sum(x, K, 0, 0.0f) / (float)K;
+    float var = chunk_tree_sum(x, K, 1, mean) / (float)K;
+    float r = sqrtf(var + eps);
     *rstd_out = 1.0f / r;
-    *mean_out = (float)mean_d;
-    if (mean_d_out) *mean_d_out = mean_d;
-    if (var_d_out) *var_d_out = var_d;
+    *mean_out = mean;
+    if (mean_d_out) *mean_d_out = (double)mean;
+    if (var_d_out) *var_d_out = (double)var;
 }
 
 /* Unfused step 1 of Fig. 2: y = fp16(LN(x)) per row.  gamma/beta may be

@@ -63,8 +63,6 @@ def _bind(lib):
     lib.zqo_quantize_weights_groupwise.argtypes = [P, I, I, I, I, P, P]
     lib.zqo_pack_int4.argtypes = [P, I, I, P]
     lib.zqo_unpack_int4.argtypes = [P, I, I, P]
-    lib.zqo_ln_exact_sums.argtypes = [P, I, P, P, P]
-    lib.zqo_ln_exact_sums.restype = None
     lib.zqo_ln_row_stats.argtypes = [P, I, ctypes.c_float, P, P, P, P]
     lib.zqo_ln_row_stats.restype = None
     lib.zqo_layernorm.argtypes = [P, P, P, I, I, ctypes.c_float, P]
@@ -139,18 +137,8 @@ def unpack_int4(packed, K: int):
     return q
 
 
-def ln_exact_sums(x):
-    """Exact S1 = sum(x*2^24), S2 = sum((x*2^24)^2) of one fp16 row, as Python ints."""
-    x = _h(x)
-    s1 = ctypes.c_int64()
-    hi = ctypes.c_uint64()
-    lo = ctypes.c_uint64()
-    _L().zqo_ln_exact_sums(_p(x), x.size, ctypes.byref(s1), ctypes.byref(hi), ctypes.byref(lo))
-    return s1.value, (hi.value << 64) | lo.value
-
-
 def ln_row_stats(x, eps: float = 1e-5):
-    """(mean fp32, rstd fp32, mean fp64, biased var fp64) of one fp16 row."""
+    """(mean fp32, rstd fp32, mean, biased var) of one fp16 row (fp32 values)."""
     x = _h(x)
     m = ctypes.c_float()
     r = ctypes.c_float()
@@ -246,6 +234,6 @@ def rounding_is_nearest() -> bool:
 
 __all__ = [
     "build", "group_of", "group_index", "quantize_weights_groupwise", "pack_int4", "unpack_int4",
-    "ln_exact_sums", "ln_row_stats", "layernorm", "token_quant", "ln_quant", "gemm_i32", "dequant",
+    "ln_row_stats", "layernorm", "token_quant", "ln_quant", "gemm_i32", "dequant",
     "linear_q", "rounding_is_nearest",
 ]

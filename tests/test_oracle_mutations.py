@@ -21,8 +21,11 @@ MUTATIONS = {
     "nibble_swap": ("packed[(size_t)o * (K / 2) + 4 * m + i] = (uint8_t)(lo | (hi << 4));",
                     "packed[(size_t)o * (K / 2) + 4 * m + i] = (uint8_t)(hi | (lo << 4));"),
     "ln_mean_sign": ("float d = h2f(x[k]) - mean;", "float d = h2f(x[k]) + mean;"),
-    "ln_var_drop_mean": ("double var_d = e2_d - msq;", "double var_d = e2_d;"),
-    "ln_unbiased_var": ("double c2 = 0x1p-48 / (double)K;", "double c2 = 0x1p-48 / (double)(K - 1);"),
+    "ln_var_drop_mean": ("float d = h2f(x[k0]) - mean;", "float d = h2f(x[k0]);"),
+    "ln_unbiased_var": ("float var = chunk_tree_sum(x, K, 1, mean) / (float)K;",
+                        "float var = chunk_tree_sum(x, K, 1, mean) / (float)(K - 1);"),
+    "ln_tree_skips_pad": ("for (int c = 0; c < n; c += 2 * step) v[c] = v[c] + v[c + step];",
+                          "for (int c = 0; c + step < n - 1; c += 2 * step) v[c] = v[c] + v[c + step];"),
     "gemm_reversed_k": ("for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];",
                         "for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[K - 1 - k];"),
     "dequant_row_scale_swapped": ("v = v * s_grp[zqo_group_of(o, N, g)];\n            v = v + (bias ? h2f(bias[o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM + dequant",

@@ -6,7 +6,9 @@
 Quantizes the weights, runs `--warmup` untimed launches and then `--reps`
 launches of the chosen kernel (the fused LN+quant of that GEMM's input, or
 the GEMM itself) recorded in one CUDA graph, printing the mean device time
-per launch measured with CUDA events around the graph replay.  Options force a GEMM variant (see zq_set_option).
+per launch measured with CUDA events around the graph replay (with --flush,
+the L2 flush before each launch is included in that time).  Options force a
+GEMM variant (see zq_set_option).
 """
 from __future__ import annotations
 
@@ -30,6 +32,8 @@ def main():
     ap.add_argument("--bn", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
+    ap.add_argument("--flush", action="store_true",
+                    help="write a 512 MB buffer before every launch (cold L2, as in bench.py)")
     a = ap.parse_args()
 
     T = a.tokens or synth.LAYERS[a.layer].tokens[0]
@@ -45,7 +49,11 @@ def main():
     Y = torch.empty((T, s.N), dtype=torch.float16, device="cuda")
     gemm = zq.gemm_w4a8 if s.bits == 4 else zq.gemm_w8a8
 
+    flush = torch.empty(128 * 1024 * 1024, dtype=torch.float32, device="cuda") if a.flush else None
+
     def run():
+        if flush is not None:
+            flush.add_(1)
         if a.kind == "gemm":
             gemm(Xq, st, Wq, sg, b, Y=Y)
         elif a.kind == "ln":

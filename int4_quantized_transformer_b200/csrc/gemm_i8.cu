@@ -59,21 +59,27 @@ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int BN_, bool WROWS_, bool W4_>
+template <int BN_, bool WROWS_, bool W4_, bool PAIR_ = false>
 struct Cfg {
   static constexpr int BN = BN_;
   static constexpr bool WROWS = WROWS_;  // weight rows on the MMA M side
   static constexpr bool W4 = W4_;
+  // CTA pair (cta_group::2): a 256 x BN tile per pair; each CTA holds 128
+  // token rows of A and BN/2 weight rows of B, and 128 rows of D in TMEM.
+  static constexpr bool PAIR = PAIR_;
+  static_assert(!PAIR || (!WROWS && !W4), "CTA pairs serve the W8A8 token-row tiling");
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // token rows per unit (token-row tiling)
   static constexpr int ACT_ROWS = WROWS ? BN : BM;
-  static constexpr int W_ROWS = WROWS ? BM : BN;
+  static constexpr int W_ROWS = WROWS ? BM : (PAIR ? BN / 2 : BN);
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK;
   static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) : 0;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
   static constexpr int STAGES_RAW =
       (kSmemBudget - (WROWS ? 0 : NUM_EPI_WARPS_C * 32 * 64) - 8 * (BN >= 64 ? BN / 2 : BN) * 8) /
       STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int EPI_ARRIVALS = PAIR ? 2 * NUM_EPI_WARPS_C : NUM_EPI_WARPS_C;
   // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
   // 32-column loads never leave the allocation.
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
@@ -100,6 +106,7 @@ struct Cfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(!PAIR || (BN / 2) % 8 == 0, "B half-tile rows must fill 8-row swizzle atoms");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -188,6 +195,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
+  // CTA pairs: rank 0 (the leader) owns the full/tempty barriers and issues
+  // the MMAs; units are numbered per pair.
+  const uint32_t crank = C::PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ustep = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], C::NUM_EPI_WARPS);
+      mbar_init(&tempty_bar[b], C::EPI_ARRIVALS);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -208,11 +220,17 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     if (!C::WROWS) tma_prefetch_desc(&map_y);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   // Set-up above touches no global memory; everything below may read what
@@ -235,14 +253,27 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       uint32_t fills[STAGES];
       for (int s = 0; s < STAGES; ++s) fills[s] = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
-        const int act_row = C::WROWS ? t.n * BN : t.m * BM;
-        const int w_row = C::WROWS ? t.m * BM : t.n * BN;
+        const int act_row = C::WROWS ? t.n * BN : t.m * C::TILE_M + static_cast<int>(crank) * BM;
+        const int w_row = C::WROWS ? t.m * BM : t.n * BN + static_cast<int>(crank) * C::W_ROWS;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status, 1)) {
             ok = false;
             break;
+          }
+          if constexpr (C::PAIR) {
+            // both CTAs' bytes complete on the leader's full barrier
+            if (crank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (act_bytes + w_bytes));
+            const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+            tma_load_2d_pair(sA + stage * C::A_BYTES, &map_act, fb, kb * BK, act_row, pol_act);
+            tma_load_2d_pair(sB + stage * C::B_BYTES, &map_w, fb, kb * BK, w_row, pol_w);
+            ++fills[stage];
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
           }
           mbar_arrive_expect_tx(&full_bar[stage], act_bytes + w_bytes);
           uint8_t* act_dst = C::WROWS ? sB + stage * C::B_BYTES : sA + stage * C::A_BYTES;
@@ -261,21 +292,24 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           }
         }
       }
-      // Drain: every copy this thread issued must land before the CTA exits.
+      // Drain: every copy issued must land before the CTA exits (for a pair,
+      // the leader's full barriers count both CTAs' copies; the follower
+      // exits only after the final cluster barrier).
       int no_abort = 0;
-      for (int s = 0; s < STAGES; ++s)
-        if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 9);
+      if (!C::PAIR || crank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 9);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_i8(BM, BN);
+    if (lane == 0 && (!C::PAIR || crank == 0)) {
+      constexpr uint32_t idesc = make_idesc_i8(C::PAIR ? 2 * BM : BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t tphase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
         if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, p.status, 2)) break;
         tc_fence_after();
@@ -292,24 +326,37 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             // advance the start address by k*32 bytes (>>4 = 2k) inside the swizzle row
-            mma_i8(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
-                   idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
+            if constexpr (C::PAIR)
+              mma_i8_pair(d_tmem, da + static_cast<uint64_t>(2 * k),
+                          db + static_cast<uint64_t>(2 * k), idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
+            else
+              mma_i8(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
+                     idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
           }
-          mma_commit(&empty_bar[stage]);
+          if constexpr (C::PAIR)
+            mma_commit_pair_mc(&empty_bar[stage], 0x3);
+          else
+            mma_commit(&empty_bar[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull_bar[buf]);
+        if constexpr (C::PAIR)
+          mma_commit_pair_mc(&tfull_bar[buf], 0x3);
+        else
+          mma_commit(&tfull_bar[buf]);
         if (++buf == 2) {
           buf = 0;
           tphase ^= 1;
         }
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      mma_commit(drain_bar);
+      if constexpr (C::PAIR)
+        mma_commit_pair_mc(drain_bar, 0x1);
+      else
+        mma_commit(drain_bar);
       int no_abort = 0;
       mbar_wait(drain_bar, 0, &no_abort, p.status, 8);
     }
@@ -330,7 +377,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     uint8_t* stg = sStg + ew * C::STG_BYTES;
     int buf = 0;
     uint32_t tphase = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+    for (int u = unit0; u < p.num_units; u += ustep) {
       const Unit t = decode_unit(u, p);
       // Scales and bias of this unit, fetched before its accumulator is ready.
       float rscale = 0.0f, rbias = 0.0f;
@@ -347,7 +394,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           colv[c] = tok < p.T ? __ldg(p.s_tok + tok) : 0.0f;
         }
       } else {
-        const int tok = t.m * BM + row_in_tile;
+        const int tok = t.m * C::TILE_M + static_cast<int>(crank) * BM + row_in_tile;
         row_idx = tok;
         if (tok < p.T) rscale = __ldg(p.s_tok + tok);
         for (int c = cb + lane; c < ce; c += 32) {
@@ -423,7 +470,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           // (rows past T / columns past N are clipped by the TMA unit): wait
           // until the previous store has read the staging buffer, write this
           // lane's 64-byte row in the 64B-swizzled layout, then issue.
-          if (o0 < p.N && t.m * BM + quad * 32 < p.T) {  // warp-uniform
+          const int row0 = t.m * C::TILE_M + static_cast<int>(crank) * BM + quad * 32;
+          if (o0 < p.N && row0 < p.T) {  // warp-uniform
             if (lane == 0) bulk_wait_group_read0();
             __syncwarp();
             const int sw = (lane >> 1) & 3;
@@ -434,7 +482,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&map_y, stg, o0, t.m * BM + quad * 32);
+              tma_store_2d(&map_y, stg, o0, row0);
               bulk_commit_group();
             }
           }
@@ -459,10 +507,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         process(a0, c0);
         if (two) process(a1, c0 + 32);
       }
-      // Release the accumulator buffer to the MMA warp.
+      // Release the accumulator buffer to the MMA warp (the leader's, for a pair).
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      if (lane == 0) {
+        if constexpr (C::PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+        else
+          mbar_arrive(&tempty_bar[buf]);
+      }
       if (++buf == 2) {
         buf = 0;
         tphase ^= 1;
@@ -522,7 +575,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!wait_warp(&full_bar[stage], phase, abort_flag, p.status, 5)) {
@@ -555,10 +608,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   if (!C::WROWS && warp >= 2 && warp < 2 + C::NUM_EPI_WARPS && lane == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync_all();  // no CTA leaves while its pair may still signal it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (C::PAIR)
+      tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -606,6 +663,7 @@ cudaError_t ensure_workspace(size_t elems, size_t counters, cudaStream_t st, Wor
 
 struct Plan {
   bool wrows;
+  bool pair;
   int bn;
   int m_tiles, n_tiles, k_blocks, splits, kb_per_split, units;
   double cost;
@@ -619,6 +677,7 @@ int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b
 Plan plan_wrows(int T, int N, int K, int sms, int forced_split) {
   Plan p{};
   p.wrows = true;
+  p.pair = false;
   int bn = 16;
   while (bn < T && bn < 256) bn *= 2;
   p.bn = bn;
@@ -649,22 +708,27 @@ Plan plan_wrows(int T, int N, int K, int sms, int forced_split) {
   return p;
 }
 
-Plan plan_trows(int T, int N, int K, int sms, int forced_bn) {
+// Token-row tiling: 128 x BN tiles per CTA, or 256 x BN tiles per CTA pair
+// (each CTA of the pair does the same MMA work as a single-CTA tile, so a
+// unit costs the same; there are half as many "slots").
+Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair) {
   Plan best{};
   best.cost = 1e30;
   const int cands[3] = {256, 192, 128};
+  const int slots = pair ? sms / 2 : sms;
   for (int bn : cands) {
     if (forced_bn && bn != forced_bn) continue;
     Plan p{};
     p.wrows = false;
+    p.pair = pair;
     p.bn = bn;
-    p.m_tiles = ceil_div(T, BM);
+    p.m_tiles = ceil_div(T, pair ? 2 * BM : BM);
     p.n_tiles = ceil_div(N, bn);
     p.k_blocks = ceil_div(K, BK);
     p.splits = 1;
     p.kb_per_split = p.k_blocks;
     p.units = p.m_tiles * p.n_tiles;
-    const int waves = ceil_div(p.units, sms);
+    const int waves = ceil_div(p.units, slots);
     p.cost = waves * (p.k_blocks * 2.0 * bn + 600.0);
     if (p.cost < best.cost) best = p;
   }
@@ -674,6 +738,7 @@ Plan plan_trows(int T, int N, int K, int sms, int forced_bn) {
 template <class C>
 cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& my,
                        const GemmParams& gp, int grid, cudaStream_t st) {
+  // grid: CTAs requested; clamped below for CTA pairs
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -684,10 +749,47 @@ cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUten
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  cudaError_t e = launch_pdl(gemm_i8_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
-                             static_cast<size_t>(C::SMEM_BYTES), st, ma, mw, my, gp);
+  if constexpr (C::PAIR) {
+    // A persistent grid of pairs larger than the number of pairs that can be
+    // resident at once would leave a second, serial wave: clamp to it.
+    static int max_pairs[64] = {};
+    if (dev >= 0 && dev < 64 && max_pairs[dev] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(C::NUM_THREADS);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_i8_kernel<C>, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1 << 20;  // unknown: keep the requested grid
+      }
+      max_pairs[dev] = n;
+    }
+    if (dev >= 0 && dev < 64) grid = std::min(grid, 2 * max_pairs[dev]);
+  }
+  cudaError_t e =
+      C::PAIR ? launch_pdl_cluster(gemm_i8_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
+                                   static_cast<size_t>(C::SMEM_BYTES), st, 2u, ma, mw, my, gp)
+              : launch_pdl(gemm_i8_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
+                           static_cast<size_t>(C::SMEM_BYTES), st, ma, mw, my, gp);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+cudaError_t dispatch_pair(int bn, const CUtensorMap& ma, const CUtensorMap& mw,
+                          const CUtensorMap& my, const GemmParams& gp, int grid, cudaStream_t st) {
+  switch (bn) {
+    case 128: return launch_cfg<Cfg<128, false, false, true>>(ma, mw, my, gp, grid, st);
+    case 192: return launch_cfg<Cfg<192, false, false, true>>(ma, mw, my, gp, grid, st);
+    default: return launch_cfg<Cfg<256, false, false, true>>(ma, mw, my, gp, grid, st);
+  }
 }
 
 template <bool WROWS, bool W4>
@@ -733,7 +835,20 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   } else {
     const int fbn = option(ZQ_OPT_GEMM_BN);
     if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
-    plan = plan_trows(T, N, K, sms, fbn);
+    // CTA pairs need less operand traffic per SM (32 KB instead of 48 KB per
+    // 128-deep K slice) but pay a cross-CTA handshake per stage and per
+    // tile.  Measured on B200 over the layer shapes: pairs of 256 x 256
+    // tiles run ~18% faster per tile when K >= 2048 and ~10% slower at small
+    // K, so the two wave-aware plans are compared with those factors.
+    const int fpair = option(ZQ_OPT_CTA_PAIR);
+    const Plan single = plan_trows(T, N, K, sms, fbn, false);
+    if (w4 || fpair == 1) {
+      plan = single;
+    } else {
+      const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true);
+      const double f = K >= 2048 ? 0.82 : 1.10;
+      plan = (fpair == 2 || pr.cost * f < single.cost) ? pr : single;
+    }
   }
 
   int* status = device_status_ptr();
@@ -769,7 +884,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   // swizzle, matching the MMA's K-major layout) or packed int4 [N][K/2]
   // (plain rows, unpacked into the swizzled layout by the kernel).
   const int act_rows = plan.wrows ? plan.bn : BM;
-  const int w_rows = plan.wrows ? BM : plan.bn;
+  const int w_rows = plan.wrows ? BM : (plan.pair ? plan.bn / 2 : plan.bn);
   CUtensorMap ma, mw, my;
   if (!encode_tma_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, T, K, BK, act_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B))
@@ -791,8 +906,14 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   int grid = std::min(plan.units, sms);
   const int cap = option(ZQ_OPT_MAX_CTAS);
   if (cap > 0) grid = std::min(grid, cap);
+  if (plan.pair) {  // CTA pairs: an even number of CTAs, one unit per pair at a time
+    grid = 2 * std::min(plan.units, sms / 2);
+    if (cap > 0) grid = std::min(grid, std::max(2, cap & ~1));
+  }
   cudaError_t e;
-  if (plan.wrows)
+  if (plan.pair)
+    e = dispatch_pair(plan.bn, ma, mw, my, gp, grid, st);
+  else if (plan.wrows)
     e = w4 ? dispatch_bn<true, true>(plan.bn, ma, mw, my, gp, grid, st)
            : dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st);
   else
@@ -883,7 +1004,7 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   } else {
     const int fbn = option(ZQ_OPT_GEMM_BN);
     if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
-    plan = plan_trows(T, N, K, sms, fbn);
+    plan = plan_trows(T, N, K, sms, fbn, false);
   }
 
   int* status = device_status_ptr();

@@ -31,6 +31,7 @@ def main():
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--bn", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
+    ap.add_argument("--pair", type=int, default=0, help="1 = single-CTA tiles, 2 = CTA pairs")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
     ap.add_argument("--flush", action="store_true",
                     help="write a 512 MB buffer before every launch (cold L2, as in bench.py)")
@@ -61,7 +62,7 @@ def main():
         else:
             zq.quantize_weights_groupwise(W, s.g, s.bits, Wq=Wq, s_grp=sg)
 
-    with zq.options(path=a.path, bn=a.bn, split_k=a.split_k):
+    with zq.options(path=a.path, bn=a.bn, split_k=a.split_k, pair=a.pair):
         for _ in range(a.warmup):
             run()
         torch.cuda.synchronize()

@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libzq.so")
 
 ZQ_OK, ZQ_ERR_NULL, ZQ_ERR_SHAPE, ZQ_ERR_ALIGN, ZQ_ERR_UNSUPPORTED, ZQ_ERR_CUDA, ZQ_ERR_TIMEOUT = range(7)
-OPT_GEMM_PATH, OPT_GEMM_BN, OPT_SPLIT_K, OPT_MAX_CTAS = 1, 2, 3, 4
+OPT_GEMM_PATH, OPT_GEMM_BN, OPT_SPLIT_K, OPT_MAX_CTAS, OPT_CTA_PAIR = 1, 2, 3, 4, 5
 
 EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
@@ -111,7 +111,7 @@ class options:
 
     def __init__(self, **kw):
         keys = {"path": OPT_GEMM_PATH, "bn": OPT_GEMM_BN, "split_k": OPT_SPLIT_K,
-                "max_ctas": OPT_MAX_CTAS}
+                "max_ctas": OPT_MAX_CTAS, "pair": OPT_CTA_PAIR}
         self.kw = {keys[k]: v for k, v in kw.items()}
 
     def __enter__(self):

@@ -167,7 +167,7 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256).
  *   ZQ_OPT_SPLIT_K     number of K splits for path 2 (1 = none).
  *   ZQ_OPT_MAX_CTAS    cap on the number of CTAs of the GEMM (persistent grid).
- *   ZQ_OPT_CTA_PAIR    path 1 with INT8 weights: 1 = one CTA per 128 x BN
+ *   ZQ_OPT_CTA_PAIR    path 1: 1 = one CTA per 128 x BN
  *                      tile, 2 = CTA pairs sharing 256 x BN tiles (tcgen05
  *                      cta_group::2); automatic picks pairs for large K.
  */

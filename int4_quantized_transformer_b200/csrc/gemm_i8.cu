@@ -67,18 +67,29 @@ struct Cfg {
   // CTA pair (cta_group::2): a 256 x BN tile per pair; each CTA holds 128
   // token rows of A and BN/2 weight rows of B, and 128 rows of D in TMEM.
   static constexpr bool PAIR = PAIR_;
-  static_assert(!PAIR || (!WROWS && !W4), "CTA pairs serve the W8A8 token-row tiling");
+  static_assert(!PAIR || !WROWS, "CTA pairs serve the token-row tiling");
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // token rows per unit (token-row tiling)
   static constexpr int ACT_ROWS = WROWS ? BN : BM;
   static constexpr int W_ROWS = WROWS ? BM : (PAIR ? BN / 2 : BN);
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK;
   static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) : 0;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
-  static constexpr int STAGES_RAW =
-      (kSmemBudget - (WROWS ? 0 : NUM_EPI_WARPS_C * 32 * 64) - 8 * (BN >= 64 ? BN / 2 : BN) * 8) /
-      STAGE_BYTES;
-  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  // Weight streaming with INT4 weights: the packed slices (with the small
+  // activation tiles) get a deep ring of their own, so that many bytes are
+  // in flight from HBM, while the unpacked weights use a shallow ring that
+  // only the unpack warps and the MMA cycle through.
+  // In this mode the deep ring holds, per K slice, the packed weights and
+  // the activation tile (B); the shallow ring holds only unpacked weights (A).
+  static constexpr bool DEEP = WROWS && W4;
+  static constexpr int FREE_BYTES =
+      kSmemBudget - (WROWS ? 0 : NUM_EPI_WARPS_C * 32 * 64) - 8 * (BN >= 64 ? BN / 2 : BN) * 8;
+  static constexpr int STAGE_BYTES = DEEP ? A_BYTES : A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int STAGES_RAW = DEEP ? 4 : FREE_BYTES / STAGE_BYTES;
+  static constexpr int STAGES_CAP = WROWS ? 12 : 8;
+  static constexpr int STAGES = STAGES_RAW > STAGES_CAP ? STAGES_CAP : STAGES_RAW;
+  static constexpr int PSTAGES_RAW =
+      DEEP ? (FREE_BYTES - STAGES * STAGE_BYTES) / (P_BYTES + B_BYTES) : STAGES;
+  static constexpr int PSTAGES = PSTAGES_RAW > 16 ? 16 : PSTAGES_RAW;  // deep (packed) ring
   static constexpr int EPI_ARRIVALS = PAIR ? 2 * NUM_EPI_WARPS_C : NUM_EPI_WARPS_C;
   // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
   // 32-column loads never leave the allocation.
@@ -91,22 +102,24 @@ struct Cfg {
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-  static constexpr int OFF_P = OFF_B + STAGES * B_BYTES;
+  static constexpr int P_RING = DEEP ? PSTAGES : STAGES;  // slots of the B and packed rings
+  static constexpr int OFF_P = OFF_B + P_RING * B_BYTES;
   // columns handled by one epilogue warp (two warps share a lane quadrant)
   static constexpr int EPI_COLS = BN >= 64 ? BN / 2 : BN;
-  static constexpr int OFF_EPI = OFF_P + STAGES * P_BYTES;           // per-warp scale/bias
+  static constexpr int OFF_EPI = OFF_P + P_RING * P_BYTES;           // per-warp scale/bias
   static constexpr int EPI_BYTES = NUM_EPI_WARPS * EPI_COLS * 2 * 4;
   // token-row tiling: per-warp staging of a 32 x 32 fp16 output block for
   // the TMA store (64-byte rows, 64-byte swizzle)
   static constexpr int STG_BYTES = WROWS ? 0 : 32 * 64;
   static constexpr int OFF_STG = ((OFF_EPI + EPI_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_BAR = OFF_STG + NUM_EPI_WARPS * STG_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 4 + 1;
+  static constexpr int NUM_BARS = 3 * STAGES + 2 * PSTAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
-  static_assert(STAGES >= 2, "not enough shared memory for two stages");
+  static_assert(STAGES >= 2 && PSTAGES >= 2, "not enough shared memory for two stages");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(!PAIR || (BN / 2) % 8 == 0, "B half-tile rows must fill 8-row swizzle atoms");
+  static_assert(!W4 || W_ROWS % 16 == 0, "unpack steps 16 rows at a time");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -186,7 +199,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* ready_bar = bars + 2 * STAGES;  // W4: unpacked operand ready
-  uint64_t* tfull_bar = bars + 3 * STAGES;  // [2]
+  uint64_t* pfull_bar = bars + 3 * STAGES;      // [PSTAGES] packed INT4 slice landed (pairs, deep ring)
+  uint64_t* pempty_bar = pfull_bar + C::PSTAGES;  // [PSTAGES] deep slot consumed by the MMA
+  uint64_t* tfull_bar = pempty_bar + C::PSTAGES;  // [2]
   uint64_t* tempty_bar = tfull_bar + 2;     // [2]
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -205,7 +220,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&ready_bar[s], C::NUM_UNPACK_WARPS > 0 ? C::NUM_UNPACK_WARPS : 1);
+      mbar_init(&ready_bar[s], C::NUM_UNPACK_WARPS > 0
+                                   ? (C::PAIR ? 2 : 1) * C::NUM_UNPACK_WARPS
+                                   : 1);
+    }
+    for (int s = 0; s < C::PSTAGES; ++s) {
+      mbar_init(&pfull_bar[s], 1);
+      mbar_init(&pempty_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
@@ -240,7 +261,40 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    if (C::DEEP && lane == 0) {
+      // packed INT4 weight slice and activation tile of each K slice into
+      // the deep ring
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_act = l2_policy_evict_last();
+      constexpr uint32_t bytes = static_cast<uint32_t>(C::P_BYTES + C::ACT_ROWS * BK);
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t fills[16];
+      for (int s = 0; s < 16; ++s) fills[s] = 0;
+      bool ok = true;
+      for (int u = unit0; ok && u < p.num_units; u += ustep) {
+        const Unit t = decode_unit(u, p);
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(&pempty_bar[stage], phase ^ 1, abort_flag, p.status, 11)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&pfull_bar[stage], bytes);
+          tma_load_2d(sP + stage * C::P_BYTES, &map_w, &pfull_bar[stage], kb * (BK / 2), t.m * BM,
+                      pol_w);
+          tma_load_2d(sB + stage * C::B_BYTES, &map_act, &pfull_bar[stage], kb * BK, t.n * BN,
+                      pol_act);
+          ++fills[stage];
+          if (++stage == C::PSTAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      int no_abort = 0;
+      for (int s = 0; s < C::PSTAGES; ++s)
+        if (fills[s]) mbar_wait(&pfull_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 12);
+    } else if (!C::DEEP && lane == 0) {
       const uint64_t pol_act = l2_policy_evict_last();
       // weights: streamed once when weight rows are the M side; in the
       // token-row tiling they are re-read by every token tile but can be far
@@ -263,11 +317,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             break;
           }
           if constexpr (C::PAIR) {
-            // both CTAs' bytes complete on the leader's full barrier
-            if (crank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (act_bytes + w_bytes));
+            // both CTAs' activation (and INT8 weight) bytes complete on the
+            // leader's full barrier; packed INT4 weights on this CTA's own
+            // pfull barrier, which its unpack warps wait on
             const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
-            tma_load_2d_pair(sA + stage * C::A_BYTES, &map_act, fb, kb * BK, act_row, pol_act);
-            tma_load_2d_pair(sB + stage * C::B_BYTES, &map_w, fb, kb * BK, w_row, pol_w);
+            if (C::W4) {
+              if (crank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * act_bytes);
+              tma_load_2d_pair(sA + stage * C::A_BYTES, &map_act, fb, kb * BK, act_row, pol_act);
+              mbar_arrive_expect_tx(&pfull_bar[stage], w_bytes);
+              tma_load_2d(sP + stage * C::P_BYTES, &map_w, &pfull_bar[stage], kb * (BK / 2), w_row,
+                          pol_w);
+            } else {
+              if (crank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * (act_bytes + w_bytes));
+              tma_load_2d_pair(sA + stage * C::A_BYTES, &map_act, fb, kb * BK, act_row, pol_act);
+              tma_load_2d_pair(sB + stage * C::B_BYTES, &map_w, fb, kb * BK, w_row, pol_w);
+            }
             ++fills[stage];
             if (++stage == STAGES) {
               stage = 0;
@@ -299,6 +363,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       if (!C::PAIR || crank == 0)
         for (int s = 0; s < STAGES; ++s)
           if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 9);
+      if (C::PAIR && C::W4)
+        for (int s = 0; s < STAGES; ++s)
+          if (fills[s]) mbar_wait(&pfull_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 10);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
@@ -306,6 +373,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       constexpr uint32_t idesc = make_idesc_i8(C::PAIR ? 2 * BM : BM, BN);
       int stage = 0;
       uint32_t phase = 0;
+      int pst = 0;  // deep ring slot (activation tile)
+      uint32_t pphase = 0;
       int buf = 0;
       uint32_t tphase = 0;
       bool ok = true;
@@ -320,9 +389,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             ok = false;
             break;
           }
+          // pairs with INT4 weights: the activations come on full, the
+          // unpacked weights of both CTAs on ready.  Deep ring: the
+          // activation tile sits in deep slot pst (landed with pfull).
+          if (C::PAIR && C::W4 && !mbar_wait(&full_bar[stage], phase, abort_flag, p.status, 6)) {
+            ok = false;
+            break;
+          }
+          if (C::DEEP && !mbar_wait(&pfull_bar[pst], pphase, abort_flag, p.status, 7)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES));
-          const uint64_t db = make_sw128_desc(smem_u32(sB + stage * C::B_BYTES));
+          const uint64_t db =
+              make_sw128_desc(smem_u32(sB + (C::DEEP ? pst : stage) * C::B_BYTES));
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             // advance the start address by k*32 bytes (>>4 = 2k) inside the swizzle row
@@ -337,6 +418,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             mma_commit_pair_mc(&empty_bar[stage], 0x3);
           else
             mma_commit(&empty_bar[stage]);
+          if constexpr (C::DEEP) {
+            mma_commit(&pempty_bar[pst]);  // the deep slot (packed + activations) is free
+            if (++pst == C::PSTAGES) {
+              pst = 0;
+              pphase ^= 1;
+            }
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -572,30 +660,58 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     // ------------------------------------------------------ INT4 unpack (W4A8)
     if constexpr (C::W4) {
       const int ut = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..127
+      const int ur = ut >> 3, uj = ut & 7;
+      const int unp_src = ur * (BK / 2) + uj * 8;
+      const int unp_dst = ur * BK + ((uj ^ (ur & 7)) << 4);
       int stage = 0;
       uint32_t phase = 0;
+      int pst = 0;  // deep ring: packed slice
+      uint32_t pphase = 0;
       bool ok = true;
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!wait_warp(&full_bar[stage], phase, abort_flag, p.status, 5)) {
+          if constexpr (C::DEEP) {
+            // the packed slice has landed, and the MMA has released the slot
+            // of the shallow ring that the unpacked weights go to
+            if (!wait_warp(&pfull_bar[pst], pphase, abort_flag, p.status, 13) ||
+                !wait_warp(&empty_bar[stage], phase ^ 1, abort_flag, p.status, 14)) {
+              ok = false;
+              break;
+            }
+          } else if (!wait_warp(C::PAIR ? &pfull_bar[stage] : &full_bar[stage], phase, abort_flag,
+                                p.status, 5)) {
             ok = false;
             break;
           }
-          const uint8_t* src = sP + stage * C::P_BYTES;
-          uint8_t* dst = C::WROWS ? sA + stage * C::A_BYTES : sB + stage * C::B_BYTES;
-#pragma unroll 4
-          for (int c = ut; c < C::W_ROWS * 8; c += 128) {
-            const int r = c >> 3, j = c & 7;
-            const uint2 pk = *reinterpret_cast<const uint2*>(src + r * (BK / 2) + j * 8);
+          // Thread ut handles 16-byte output chunk j = ut % 8 of rows
+          // r = ut / 8 + 16 i: stepping 16 rows keeps r % 8, hence the
+          // swizzled chunk position, fixed, so the shared-memory offsets are
+          // per-thread constants plus i * (16 rows).
+          const uint8_t* src = sP + (C::DEEP ? pst : stage) * C::P_BYTES + unp_src;
+          uint8_t* dst = (C::WROWS ? sA + stage * C::A_BYTES : sB + stage * C::B_BYTES) + unp_dst;
+#pragma unroll
+          for (int i = 0; i < C::W_ROWS / 16; ++i) {
+            const uint2 pk = *reinterpret_cast<const uint2*>(src + i * 16 * (BK / 2));
             uint4 o;
             unpack8_x16(pk.x, o.x, o.y);
             unpack8_x16(pk.y, o.z, o.w);
-            *reinterpret_cast<uint4*>(dst + r * BK + ((j ^ (r & 7)) << 4)) = o;
+            *reinterpret_cast<uint4*>(dst + i * 16 * BK) = o;
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ready_bar[stage]);
+          if (lane == 0) {
+            if constexpr (C::PAIR)
+              mbar_arrive_cluster(mapa_shared(smem_u32(&ready_bar[stage]), 0));
+            else
+              mbar_arrive(&ready_bar[stage]);
+          }
+          if constexpr (C::DEEP) {
+            if (++pst == C::PSTAGES) {
+              pst = 0;
+              pphase ^= 1;
+            }
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -783,12 +899,13 @@ cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUten
   return cudaGetLastError();
 }
 
+template <bool W4>
 cudaError_t dispatch_pair(int bn, const CUtensorMap& ma, const CUtensorMap& mw,
                           const CUtensorMap& my, const GemmParams& gp, int grid, cudaStream_t st) {
   switch (bn) {
-    case 128: return launch_cfg<Cfg<128, false, false, true>>(ma, mw, my, gp, grid, st);
-    case 192: return launch_cfg<Cfg<192, false, false, true>>(ma, mw, my, gp, grid, st);
-    default: return launch_cfg<Cfg<256, false, false, true>>(ma, mw, my, gp, grid, st);
+    case 128: return launch_cfg<Cfg<128, false, W4, true>>(ma, mw, my, gp, grid, st);
+    case 192: return launch_cfg<Cfg<192, false, W4, true>>(ma, mw, my, gp, grid, st);
+    default: return launch_cfg<Cfg<256, false, W4, true>>(ma, mw, my, gp, grid, st);
   }
 }
 
@@ -842,11 +959,13 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
     // K, so the two wave-aware plans are compared with those factors.
     const int fpair = option(ZQ_OPT_CTA_PAIR);
     const Plan single = plan_trows(T, N, K, sms, fbn, false);
-    if (w4 || fpair == 1) {
+    if (fpair == 1) {
       plan = single;
     } else {
       const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true);
-      const double f = K >= 2048 ? 0.82 : 1.10;
+      // INT4: the unpack stage, not the operand feed, bounds the mainloop;
+      // pairs measured slower there, so they are used only when forced.
+      const double f = w4 ? 1e9 : (K >= 2048 ? 0.82 : 1.10);
       plan = (fpair == 2 || pr.cost * f < single.cost) ? pr : single;
     }
   }
@@ -912,7 +1031,8 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   }
   cudaError_t e;
   if (plan.pair)
-    e = dispatch_pair(plan.bn, ma, mw, my, gp, grid, st);
+    e = w4 ? dispatch_pair<true>(plan.bn, ma, mw, my, gp, grid, st)
+           : dispatch_pair<false>(plan.bn, ma, mw, my, gp, grid, st);
   else if (plan.wrows)
     e = w4 ? dispatch_bn<true, true>(plan.bn, ma, mw, my, gp, grid, st)
            : dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st);

@@ -182,14 +182,16 @@ def test_gemm_token_rows_tiles(zq, bits, bn, T, N, K):
     _check_gemm(zq, T, N, K, 8, bits, seed=bn, path=1, bn=bn, pair=1)
 
 
+@pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("bn", [128, 192, 256])
 @pytest.mark.parametrize("T,N,K", [(16, 256, 64), (300, 1000, 512), (1024, 768, 1024),
                                    (513, 2304, 768)])
-def test_gemm_cta_pair_tiles(zq, bn, T, N, K):
+def test_gemm_cta_pair_tiles(zq, bits, bn, T, N, K):
     """256-row tiles shared by a CTA pair (tcgen05 cta_group::2): each CTA
-    loads 128 token rows and half of the weight rows; ragged token counts
-    leave the second CTA's rows partly or wholly past T."""
-    _check_gemm(zq, T, N, K, 8, 8, seed=bn + 1, path=1, bn=bn, pair=2)
+    loads 128 token rows and half of the weight rows (INT4: and unpacks its
+    half); ragged token counts leave the second CTA's rows partly or wholly
+    past T."""
+    _check_gemm(zq, T, N, K, 8, bits, seed=bn + 1, path=1, bn=bn, pair=2)
 
 
 @pytest.mark.parametrize("bits", [8, 4])
@@ -207,6 +209,7 @@ def test_gemm_persistent_loop_with_few_ctas(zq):
     _check_gemm(zq, 640, 1024, 512, 8, 4, seed=4, path=1, bn=256, max_ctas=3)
     _check_gemm(zq, 1280, 1024, 512, 8, 8, seed=6, path=1, bn=128, max_ctas=4, pair=2)
     _check_gemm(zq, 1000, 2048, 384, 8, 8, seed=7, path=1, bn=256, max_ctas=6, pair=2)
+    _check_gemm(zq, 1000, 2048, 384, 8, 4, seed=8, path=1, bn=256, max_ctas=6, pair=2)
     _check_gemm(zq, 16, 2048, 1024, 8, 8, seed=5, path=2, split_k=4, max_ctas=7)
 
 

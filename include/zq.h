@@ -103,8 +103,9 @@ zq_status zq_ln_quant(const void* X, const void* gamma, const void* beta, int T,
  *               Y[t][o] = fp16(((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]))
  *   acc_dbg     int32 [T][N] or NULL: also store acc (for checking).
  * Runs on tcgen05 tensor cores.  Small T (weight-streaming) shapes split K
- * across SMs and reduce the exact int32 partial sums in a library-owned
- * workspace; calls that use it on different streams must not overlap.
+ * across SMs: the exact int32 partial sums go to a library-owned workspace
+ * and a second kernel on the same stream adds them and dequantizes; calls
+ * that use the workspace on different streams must not overlap.
  * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
  * 16 <= K <= 133136, K % 16 == 0 (so that 127*127*K < 2^31), 1 <= g <= N,
  * pointers 16-byte aligned.
@@ -134,17 +135,17 @@ zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
  *   Same arguments, results and requirements as zq_gemm_w8a8.  The caller
  *   still owns and passes every input and output.  The scratch memory of the
  *   split-K reduction (small token counts) comes from a fixed array of
- *   8 MiB + 64 KiB in device memory that the library declares statically;
- *   every GPU that loads the library holds it until the process exits, and
- *   no call of this function allocates or frees anything.
+ *   8 MiB in device memory that the library declares statically; every GPU
+ *   that loads the library holds it until the process exits, and no call of
+ *   this function allocates or frees anything.
  *   Limit: when the planned split-K reduction needs more than that, i.e.
- *   splits * T * N int32 partial sums above 8 MiB, or more than 16384 tile
- *   counters, the call returns ZQ_ERR_SHAPE without launching.
+ *   splits * T * N int32 partial sums above 8 MiB, the call returns
+ *   ZQ_ERR_SHAPE without launching.
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
  *   All calls on a device share the one array: calls whose work may overlap
  *   on the GPU (for example on different streams) race on it and give wrong
- *   results.  Each call clears the counters it uses, on `stream`.
+ *   results.
  */
 zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
                                const float* s_grp, int g, const void* bias, int T, int N, int K,

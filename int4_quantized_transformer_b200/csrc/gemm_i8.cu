@@ -11,12 +11,16 @@
 //  * weight rows on the MMA M side (small T, weight-streaming, HBM-bound):
 //    128 output features x all tokens (padded to BN in {16..256}) per unit,
 //    with K split across SMs when there are fewer weight tiles than SMs.
-//    Integer partial sums are added exactly (red.add.s32) into a workspace;
-//    the last split of each tile (a per-tile counter) applies the dequant.
+//    Each split stores its exact int32 partial sums into a workspace; a
+//    small second kernel, chained with programmatic dependent launch, adds
+//    the splits (exact) and applies the dequant.  The mainloop never waits
+//    on the reduction.
 //
 // Warp roles (one CTA per SM):
 //   warp 0     TMA producer: activation and weight tiles, 128-byte K slices,
-//              128B-swizzled, into a STAGES-deep mbarrier ring;
+//              128B-swizzled, into a STAGES-deep mbarrier ring (with weight
+//              rows on M, the last warp is a second producer: the two take
+//              alternate K slices);
 //   warp 1     TMEM allocator and MMA issuer: tcgen05.mma kind::i8, M=128,
 //              N=BN, K=32, int32 accumulators in TMEM (two buffers, so the
 //              epilogue of one unit overlaps the mainloop of the next);
@@ -81,23 +85,38 @@ struct Cfg {
   // In this mode the deep ring holds, per K slice, the packed weights and
   // the activation tile (B); the shallow ring holds only unpacked weights (A).
   static constexpr bool DEEP = WROWS && W4;
+  // Weight streaming is bound by how fast TMA copies are issued: one issuing
+  // thread per SM keeps well under the HBM bandwidth in flight, two do not.
+  // The second producer warp is the last warp of the CTA; the producers take
+  // alternate K slices, and the rings have an even number of slots so that
+  // each slot is only ever filled by one of them.
+  static constexpr int NUM_PROD_WARPS = WROWS ? 2 : 1;
   static constexpr int FREE_BYTES =
       kSmemBudget - (WROWS ? 0 : NUM_EPI_WARPS_C * 32 * 64) - 8 * (BN >= 64 ? BN / 2 : BN) * 8;
   static constexpr int STAGE_BYTES = DEEP ? A_BYTES : A_BYTES + B_BYTES + P_BYTES;
   static constexpr int STAGES_RAW = DEEP ? 4 : FREE_BYTES / STAGE_BYTES;
   static constexpr int STAGES_CAP = WROWS ? 12 : 8;
-  static constexpr int STAGES = STAGES_RAW > STAGES_CAP ? STAGES_CAP : STAGES_RAW;
+  static constexpr int STAGES_ANY = STAGES_RAW > STAGES_CAP ? STAGES_CAP : STAGES_RAW;
+  static constexpr int STAGES = NUM_PROD_WARPS == 2 ? STAGES_ANY & ~1 : STAGES_ANY;
   static constexpr int PSTAGES_RAW =
       DEEP ? (FREE_BYTES - STAGES * STAGE_BYTES) / (P_BYTES + B_BYTES) : STAGES;
-  static constexpr int PSTAGES = PSTAGES_RAW > 16 ? 16 : PSTAGES_RAW;  // deep (packed) ring
+  static constexpr int PSTAGES_ANY = PSTAGES_RAW > 16 ? 16 : PSTAGES_RAW;
+  static constexpr int PSTAGES = DEEP ? PSTAGES_ANY & ~1 : PSTAGES_ANY;  // deep (packed) ring
   static constexpr int EPI_ARRIVALS = PAIR ? 2 * NUM_EPI_WARPS_C : NUM_EPI_WARPS_C;
   // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
   // 32-column loads never leave the allocation.
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
-  static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_STRIDE);
+  // With weight rows on M the tokens are few (N = BN is small), so one
+  // tcgen05.mma is short and successive MMAs into one accumulator form a
+  // dependent chain whose latency, not the data, sets the pace.  The K steps
+  // of a slice rotate over NACC independent accumulators instead; the
+  // epilogue adds them (exact int32 sums).
+  static constexpr int NACC = WROWS ? (BN <= 64 ? 4 : (BN <= 128 ? 2 : 1)) : 1;
+  static constexpr int BUF_COLS = NACC * ACC_STRIDE;  // TMEM columns per accumulator buffer
+  static constexpr int TMEM_COLS = pow2_at_least(2 * BUF_COLS);
   static constexpr int NUM_EPI_WARPS = NUM_EPI_WARPS_C;
   static constexpr int NUM_UNPACK_WARPS = W4 ? 4 : 0;
-  static constexpr int NUM_WARPS = 2 + NUM_EPI_WARPS + NUM_UNPACK_WARPS;
+  static constexpr int NUM_WARPS = 1 + NUM_PROD_WARPS + NUM_EPI_WARPS + NUM_UNPACK_WARPS;
   static constexpr int NUM_THREADS = 32 * NUM_WARPS;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
   static constexpr int OFF_A = 0;
@@ -117,10 +136,14 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGES >= 2 && PSTAGES >= 2, "not enough shared memory for two stages");
+  static_assert(NUM_PROD_WARPS == 1 || (STAGES % 2 == 0 && (!DEEP || PSTAGES % 2 == 0)),
+                "two producers need rings with an even number of slots");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(!PAIR || (BN / 2) % 8 == 0, "B half-tile rows must fill 8-row swizzle atoms");
-  static_assert(!W4 || W_ROWS % 16 == 0, "unpack steps 16 rows at a time");
+  static_assert(!W4 || (W_ROWS % (4 * NUM_UNPACK_WARPS) == 0 && (4 * NUM_UNPACK_WARPS) % 8 == 0),
+                "unpack steps keep the row's swizzle phase");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+  static_assert(TMEM_COLS <= 512 && (BK / UMMA_K) % NACC == 0, "TMEM accumulators");
 };
 
 struct GemmParams {
@@ -130,7 +153,6 @@ struct GemmParams {
   __half* Y;
   int32_t* acc_dbg;
   int32_t* ws;     // split-K partial sums [splits][T][N]
-  int* counters;   // split-K arrival counts, [m_tiles*n_tiles*8] (zero between calls)
   int* status;
   int T, N, K, g;
   int m_tiles, n_tiles, k_blocks, splits, kb_per_split, num_units;
@@ -259,8 +281,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   grid_dependency_wait();
   grid_launch_dependents();
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == 0 || (C::NUM_PROD_WARPS == 2 && warp == C::NUM_WARPS - 1)) {
+    // ------------------------------------------------------ TMA producer(s)
+    // With two producers, producer `pid` issues the K slices whose running
+    // index is congruent to pid modulo 2; both walk the same units and ring.
+    constexpr int NP = C::NUM_PROD_WARPS;
+    const int pid = warp == 0 ? 0 : 1;
+    int seq = 0;
     if (C::DEEP && lane == 0) {
       // packed INT4 weight slice and activation tile of each K slice into
       // the deep ring
@@ -275,6 +302,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (NP > 1 && (seq++ % NP) != pid) {
+            if (++stage == C::PSTAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           if (!mbar_wait(&pempty_bar[stage], phase ^ 1, abort_flag, p.status, 11)) {
             ok = false;
             break;
@@ -312,6 +346,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         const int act_row = C::WROWS ? t.n * BN : t.m * C::TILE_M + static_cast<int>(crank) * BM;
         const int w_row = C::WROWS ? t.m * BM : t.n * BN + static_cast<int>(crank) * C::W_ROWS;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (NP > 1 && (seq++ % NP) != pid) {
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status, 1)) {
             ok = false;
             break;
@@ -382,7 +423,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         const Unit t = decode_unit(u, p);
         if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, p.status, 2)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::ACC_STRIDE);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::BUF_COLS);
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           uint64_t* rb = C::W4 ? &ready_bar[stage] : &full_bar[stage];
           if (!mbar_wait(rb, phase, abort_flag, p.status, 3)) {
@@ -411,8 +452,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
               mma_i8_pair(d_tmem, da + static_cast<uint64_t>(2 * k),
                           db + static_cast<uint64_t>(2 * k), idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
             else
-              mma_i8(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
-                     idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
+              mma_i8(d_tmem + static_cast<uint32_t>((k % C::NACC) * C::ACC_STRIDE),
+                     da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), idesc,
+                     (kb > t.kb0 || k >= C::NACC) ? 1u : 0u);
           }
           if constexpr (C::PAIR)
             mma_commit_pair_mc(&empty_bar[stage], 0x3);
@@ -467,17 +509,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     uint32_t tphase = 0;
     for (int u = unit0; u < p.num_units; u += ustep) {
       const Unit t = decode_unit(u, p);
-      // Scales and bias of this unit, fetched before its accumulator is ready.
+      // Scales and bias of this unit, fetched before its accumulator is ready
+      // (a K split of the weight-row tiling stores raw partial sums and needs
+      // none of them).
+      const bool split = C::WROWS && p.splits > 1;
       float rscale = 0.0f, rbias = 0.0f;
       int row_idx;
       if (C::WROWS) {
         const int o = t.m * BM + row_in_tile;
         row_idx = o;
-        if (o < p.N) {
+        if (o < p.N && !split) {
           rscale = __ldg(p.s_grp + group_of(o, p.N, p.g));
           rbias = p.bias ? __half2float(p.bias[o]) : 0.0f;
         }
-        for (int c = cb + lane; c < ce; c += 32) {
+        for (int c = cb + lane; c < ce && !split; c += 32) {
           const int tok = t.n * BN + c;
           colv[c] = tok < p.T ? __ldg(p.s_tok + tok) : 0.0f;
         }
@@ -495,8 +540,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       if (!wait_warp(&tfull_bar[buf], tphase, abort_flag, p.status, 4)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                             static_cast<uint32_t>(buf * C::ACC_STRIDE);
-      const bool split = C::WROWS && p.splits > 1;
+                             static_cast<uint32_t>(buf * C::BUF_COLS);
 
       auto process = [&](const uint32_t (&acc)[32], int c0) {
         if (C::WROWS) {
@@ -577,6 +621,30 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         }
       };
 
+      if constexpr (C::NACC > 1) {
+        // 32 columns at a time: the NACC partial accumulators, added
+#pragma unroll 1
+        for (int c0 = cb; c0 < ce; c0 += 32) {
+          uint32_t a0[32], b0[32];
+          tmem_ld_32x32b_x32(t_row + c0, a0);
+          tmem_ld_32x32b_x32(t_row + C::ACC_STRIDE + c0, b0);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) a0[j] += b0[j];
+#pragma unroll 1
+          for (int a = 2; a < C::NACC; ++a) {
+            tmem_ld_32x32b_x32(t_row + a * C::ACC_STRIDE + c0, b0);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a0[j] += b0[j];
+          }
+          if (C::W4) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
+          }
+          process(a0, c0);
+        }
+      } else {
       // Two 32-column TMEM loads in flight before each wait.
 #pragma unroll 1
       for (int c0 = cb; c0 < ce; c0 += 64) {
@@ -595,6 +663,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         process(a0, c0);
         if (two) process(a1, c0 + 32);
       }
+      }
       // Release the accumulator buffer to the MMA warp (the leader's, for a pair).
       tc_fence_before();
       __syncwarp();
@@ -608,58 +677,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         buf = 0;
         tphase ^= 1;
       }
-      if (split && cb < ce) {
-        // The last of the splits of this tile finalises its (quadrant, column
-        // half): the exact int32 partial sums of all splits -> dequant -> fp16.
-        __threadfence();
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          int* ctr = p.counters + (((t.n * p.m_tiles + t.m) * 4 + quad) * 2 + half);
-          last = (atomicAdd(ctr, 1) == p.splits - 1) ? 1 : 0;
-          if (last) *ctr = 0;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          const int o = row_idx;
-          if (o < p.N) {
-            const size_t plane = static_cast<size_t>(p.T) * p.N;
-            // eight token columns at a time, so the partial-sum loads of all
-            // splits are independent and in flight together
-            for (int c = cb; c < ce && t.n * BN + c < p.T; c += 8) {
-              int a[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) a[j] = 0;
-              for (int sp = 0; sp < p.splits; ++sp) {
-                const int32_t* src = p.ws + sp * plane + o;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                  const int tok = t.n * BN + c + j;
-                  if (c + j < ce && tok < p.T) a[j] += __ldcg(src + static_cast<size_t>(tok) * p.N);
-                }
-              }
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int tok = t.n * BN + c + j;
-                if (c + j < ce && tok < p.T) {
-                  const size_t idx = static_cast<size_t>(tok) * p.N + o;
-                  float v = __fmul_rn(__int2float_rn(a[j]), colv[c + j]);
-                  v = __fadd_rn(__fmul_rn(v, rscale), rbias);
-                  p.Y[idx] = __float2half_rn(v);
-                  if (p.acc_dbg) p.acc_dbg[idx] = a[j];
-                }
-              }
-            }
-          }
-        }
-      }
       __syncwarp();
     }
   } else {
     // ------------------------------------------------------ INT4 unpack (W4A8)
     if constexpr (C::W4) {
-      const int ut = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0..127
+      const int ut = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0 .. 32*NUM_UNPACK_WARPS-1
+      constexpr int UROWS = 4 * C::NUM_UNPACK_WARPS;  // rows of one unpack step
       const int ur = ut >> 3, uj = ut & 7;
       const int unp_src = ur * (BK / 2) + uj * 8;
       const int unp_dst = ur * BK + ((uj ^ (ur & 7)) << 4);
@@ -685,18 +709,18 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             break;
           }
           // Thread ut handles 16-byte output chunk j = ut % 8 of rows
-          // r = ut / 8 + 16 i: stepping 16 rows keeps r % 8, hence the
-          // swizzled chunk position, fixed, so the shared-memory offsets are
-          // per-thread constants plus i * (16 rows).
+          // r = ut / 8 + UROWS i: stepping a multiple of 8 rows keeps r % 8,
+          // hence the swizzled chunk position, fixed, so the shared-memory
+          // offsets are per-thread constants plus i * (UROWS rows).
           const uint8_t* src = sP + (C::DEEP ? pst : stage) * C::P_BYTES + unp_src;
           uint8_t* dst = (C::WROWS ? sA + stage * C::A_BYTES : sB + stage * C::B_BYTES) + unp_dst;
 #pragma unroll
-          for (int i = 0; i < C::W_ROWS / 16; ++i) {
-            const uint2 pk = *reinterpret_cast<const uint2*>(src + i * 16 * (BK / 2));
+          for (int i = 0; i < C::W_ROWS / UROWS; ++i) {
+            const uint2 pk = *reinterpret_cast<const uint2*>(src + i * UROWS * (BK / 2));
             uint4 o;
             unpack8_x16(pk.x, o.x, o.y);
             unpack8_x16(pk.y, o.z, o.w);
-            *reinterpret_cast<uint4*>(dst + i * 16 * BK) = o;
+            *reinterpret_cast<uint4*>(dst + i * UROWS * BK) = o;
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -735,18 +759,63 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   }
 }
 
+// Split-K finalisation for the weight-row tiling: sum the int32 partial
+// sums of the K splits (exact) and dequantize, eight outputs per thread:
+// y = fp16(((f32(acc) * s_tok[t]) * s_grp[group(o)]) + f32(bias[o])).
+__global__ void __launch_bounds__(256)
+    splitk_finalize_kernel(const int32_t* __restrict__ ws, int splits, const float* __restrict__ s_tok,
+                           const float* __restrict__ s_grp, const __half* __restrict__ bias,
+                           __half* __restrict__ Y, int32_t* __restrict__ acc_dbg, int T, int N,
+                           int g) {
+  // the partial sums are written by the GEMM kernel just before this one
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const size_t plane = static_cast<size_t>(T) * N;
+  const size_t n8 = plane / 8;  // N % 8 == 0
+  for (size_t v = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; v < n8;
+       v += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t idx = v * 8;
+    const int t = static_cast<int>(idx / N);
+    const int o = static_cast<int>(idx - static_cast<size_t>(t) * N);
+    int4 lo = __ldcg(reinterpret_cast<const int4*>(ws + idx));
+    int4 hi = __ldcg(reinterpret_cast<const int4*>(ws + idx) + 1);
+    for (int sp = 1; sp < splits; ++sp) {
+      const int4* src = reinterpret_cast<const int4*>(ws + sp * plane + idx);
+      const int4 a = __ldcg(src), b = __ldcg(src + 1);
+      lo.x += a.x; lo.y += a.y; lo.z += a.z; lo.w += a.w;
+      hi.x += b.x; hi.y += b.y; hi.z += b.z; hi.w += b.w;
+    }
+    const int acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const float st = __ldg(s_tok + t);
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      float v0 = __fmul_rn(__int2float_rn(acc[j]), st);
+      float v1 = __fmul_rn(__int2float_rn(acc[j + 1]), st);
+      v0 = __fadd_rn(__fmul_rn(v0, __ldg(s_grp + group_of(o + j, N, g))),
+                     bias ? __half2float(bias[o + j]) : 0.0f);
+      v1 = __fadd_rn(__fmul_rn(v1, __ldg(s_grp + group_of(o + j + 1, N, g))),
+                     bias ? __half2float(bias[o + j + 1]) : 0.0f);
+      h[j / 2] = pack_half2(v0, v1);
+    }
+    *reinterpret_cast<uint4*>(Y + idx) = make_uint4(h[0], h[1], h[2], h[3]);
+    if (acc_dbg) {
+      reinterpret_cast<int4*>(acc_dbg + idx)[0] = lo;
+      reinterpret_cast<int4*>(acc_dbg + idx)[1] = hi;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host
 
 struct Workspace {
   int32_t* ws = nullptr;
   size_t ws_elems = 0;
-  int* counters = nullptr;
-  size_t counter_elems = 0;
 };
 std::mutex g_ws_mu;
 Workspace g_ws[64];
 
-cudaError_t ensure_workspace(size_t elems, size_t counters, cudaStream_t st, Workspace** out) {
+cudaError_t ensure_workspace(size_t elems, Workspace** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -759,22 +828,21 @@ cudaError_t ensure_workspace(size_t elems, size_t counters, cudaStream_t st, Wor
     w.ws_elems = 0;
     e = cudaMalloc(&w.ws, elems * sizeof(int32_t));
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(w.ws, 0, elems * sizeof(int32_t), st);
-    if (e != cudaSuccess) return e;
     w.ws_elems = elems;
-  }
-  if (w.counter_elems < counters) {
-    if (w.counters) cudaFree(w.counters);
-    w.counters = nullptr;
-    w.counter_elems = 0;
-    e = cudaMalloc(&w.counters, counters * sizeof(int));
-    if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(w.counters, 0, counters * sizeof(int), st);
-    if (e != cudaSuccess) return e;
-    w.counter_elems = counters;
   }
   *out = &w;
   return cudaSuccess;
+}
+
+// The split-K finalisation, launched right after the GEMM kernel on the same
+// stream (programmatic dependent launch: it is scheduled early and waits in
+// the kernel for the GEMM's partial sums).
+cudaError_t launch_finalize(const GemmParams& gp, cudaStream_t st) {
+  const size_t n8 = static_cast<size_t>(gp.T) * gp.N / 8;
+  const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 4 * 148));
+  return launch_pdl(splitk_finalize_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, st,
+                    static_cast<const int32_t*>(gp.ws), gp.splits, gp.s_tok, gp.s_grp, gp.bias,
+                    gp.Y, gp.acc_dbg, gp.T, gp.N, gp.g);
 }
 
 struct Plan {
@@ -992,11 +1060,9 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   gp.num_units = plan.units;
   if (plan.wrows && plan.splits > 1) {
     Workspace* w = nullptr;
-    const size_t counters = static_cast<size_t>(plan.m_tiles) * plan.n_tiles * 8;
-    if (ensure_workspace(static_cast<size_t>(plan.splits) * T * N, counters, st, &w) != cudaSuccess)
+    if (ensure_workspace(static_cast<size_t>(plan.splits) * T * N, &w) != cudaSuccess)
       return ZQ_ERR_CUDA;
     gp.ws = w->ws;
-    gp.counters = w->counters;
   }
 
   // TMA descriptors: int8 activations [T][K]; weights int8 [N][K] (128B
@@ -1039,6 +1105,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   else
     e = w4 ? dispatch_bn<false, true>(plan.bn, ma, mw, my, gp, grid, st)
            : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
+  if (e == cudaSuccess && plan.wrows && plan.splits > 1) e = launch_finalize(gp, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 
@@ -1061,7 +1128,7 @@ extern "C" zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const ui
 // Allocation-free variant of zq_gemm_w8a8.
 //
 // The split-K reduction of the weight-streaming tiling needs scratch memory
-// (one int32 partial-sum slice per K split plus per-tile arrival counters).
+// (one int32 partial-sum slice per K split).
 // zq_gemm_w8a8 allocates that lazily with cudaMalloc.  Some callers cannot
 // let a library allocate: a serving runtime that owns the whole device
 // memory pool, a process whose memory budget is fixed up front, or code that
@@ -1073,9 +1140,8 @@ namespace zq {
 namespace {
 
 constexpr size_t kNoAllocPartialInts = (8u << 20) / sizeof(int32_t);  // 8 MiB of partial sums
-constexpr size_t kNoAllocCounters = 16384;                           // 64 KiB of counters
 
-static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocPartialInts + kNoAllocCounters];
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocPartialInts];
 
 std::mutex g_noalloc_mu;
 int32_t* g_noalloc_ptr[64] = {};
@@ -1149,16 +1215,11 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   gp.num_units = plan.units;
   if (plan.wrows && plan.splits > 1) {
     const size_t partial = static_cast<size_t>(plan.splits) * T * N;
-    const size_t counters = static_cast<size_t>(plan.m_tiles) * plan.n_tiles * 8;
-    if (partial > kNoAllocPartialInts || counters > kNoAllocCounters) return ZQ_ERR_SHAPE;
+    if (partial > kNoAllocPartialInts) return ZQ_ERR_SHAPE;
     int32_t* scratch = nullptr;
     if (noalloc_scratch(&scratch) != cudaSuccess) return ZQ_ERR_CUDA;
-    // The arrival counters must start at zero; the array keeps whatever the
-    // previous call left there.  The partial sums need no clearing.
-    int* ctr = reinterpret_cast<int*>(scratch + kNoAllocPartialInts);
-    if (cudaMemsetAsync(ctr, 0, counters * sizeof(int), st) != cudaSuccess) return ZQ_ERR_CUDA;
+    // every partial sum the finalisation reads is written by this call
     gp.ws = scratch;
-    gp.counters = ctr;
   }
 
   const int act_rows = plan.wrows ? plan.bn : BM;
@@ -1177,7 +1238,8 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   int grid = std::min(plan.units, sms);
   const int cap = option(ZQ_OPT_MAX_CTAS);
   if (cap > 0) grid = std::min(grid, cap);
-  const cudaError_t e = plan.wrows ? dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st)
-                                   : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
+  cudaError_t e = plan.wrows ? dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st)
+                             : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
+  if (e == cudaSuccess && plan.wrows && plan.splits > 1) e = launch_finalize(gp, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }

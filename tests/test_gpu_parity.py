@@ -24,6 +24,16 @@ def zq():
     assert rc == m.ZQ_OK, f"device status {rc} detail {detail}"
 
 
+@pytest.fixture(autouse=True)
+def _device_status_clean(zq):
+    """Every test leaves the device status word clean: a bounded wait that
+    ran out anywhere (a drain at kernel exit included) fails the test that
+    launched it, even when its outputs were right."""
+    yield
+    rc, detail = zq.device_status()
+    assert rc == zq.ZQ_OK, f"device status {rc} ({zq.status_str(rc)}), wait site {detail}"
+
+
 def dev(t):
     return t.cuda()
 

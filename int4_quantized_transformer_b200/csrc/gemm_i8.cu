@@ -91,8 +91,13 @@ struct Cfg {
   // alternate K slices, and the rings have an even number of slots so that
   // each slot is only ever filled by one of them.
   static constexpr int NUM_PROD_WARPS = WROWS ? 2 : 1;
+  // columns handled by one epilogue warp (two warps share a lane quadrant)
+  static constexpr int EPI_COLS = BN >= 64 ? BN / 2 : BN;
+  // token-row tiling: per-warp staging of a 32 x 32 fp16 output block for
+  // the TMA store (64-byte rows, 64-byte swizzle)
+  static constexpr int STG_BYTES = WROWS ? 0 : 32 * 32 * 2;
   static constexpr int FREE_BYTES =
-      kSmemBudget - (WROWS ? 0 : NUM_EPI_WARPS_C * 32 * 64) - 8 * (BN >= 64 ? BN / 2 : BN) * 8;
+      kSmemBudget - NUM_EPI_WARPS_C * STG_BYTES - 8 * EPI_COLS * 8;
   static constexpr int STAGE_BYTES = DEEP ? A_BYTES : A_BYTES + B_BYTES + P_BYTES;
   static constexpr int STAGES_RAW = DEEP ? 4 : FREE_BYTES / STAGE_BYTES;
   static constexpr int STAGES_CAP = WROWS ? 12 : 8;
@@ -123,13 +128,8 @@ struct Cfg {
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int P_RING = DEEP ? PSTAGES : STAGES;  // slots of the B and packed rings
   static constexpr int OFF_P = OFF_B + P_RING * B_BYTES;
-  // columns handled by one epilogue warp (two warps share a lane quadrant)
-  static constexpr int EPI_COLS = BN >= 64 ? BN / 2 : BN;
   static constexpr int OFF_EPI = OFF_P + P_RING * P_BYTES;           // per-warp scale/bias
   static constexpr int EPI_BYTES = NUM_EPI_WARPS * EPI_COLS * 2 * 4;
-  // token-row tiling: per-warp staging of a 32 x 32 fp16 output block for
-  // the TMA store (64-byte rows, 64-byte swizzle)
-  static constexpr int STG_BYTES = WROWS ? 0 : 32 * 64;
   static constexpr int OFF_STG = ((OFF_EPI + EPI_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_BAR = OFF_STG + NUM_EPI_WARPS * STG_BYTES;
   static constexpr int NUM_BARS = 3 * STAGES + 2 * PSTAGES + 4 + 1;
@@ -144,6 +144,7 @@ struct Cfg {
                 "unpack steps keep the row's swizzle phase");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(TMEM_COLS <= 512 && (BK / UMMA_K) % NACC == 0, "TMEM accumulators");
+  static_assert(EPI_COLS <= 128, "epilogue prefetch holds at most four columns per lane");
 };
 
 struct GemmParams {
@@ -507,36 +508,69 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     uint8_t* stg = sStg + ew * C::STG_BYTES;
     int buf = 0;
     uint32_t tphase = 0;
-    for (int u = unit0; u < p.num_units; u += ustep) {
+    // A K split of the weight-row tiling stores raw partial sums and needs no
+    // scales or bias.
+    const bool split = C::WROWS && p.splits > 1;
+    // The scales and bias of a unit are loaded into registers one unit ahead,
+    // so their global-load latency overlaps the previous unit's epilogue
+    // ("read the two groups of quantization scales in advance").  Lane l
+    // holds columns cb + l + 32 i.
+    constexpr int PCOLS = (C::EPI_COLS + 31) / 32;
+    // bias stays in its fp16 form until used, so that nothing waits on the load
+    float n_rs = 0.0f, n_cv[PCOLS];
+    __half n_rb, n_cb[PCOLS];
+    auto fetch = [&](int u) {
+      n_rs = 0.0f;
+      n_rb = __float2half_rn(0.0f);
+#pragma unroll
+      for (int i = 0; i < PCOLS; ++i) {
+        n_cv[i] = 0.0f;
+        n_cb[i] = __float2half_rn(0.0f);
+      }
+      if (u >= p.num_units || split) return;
       const Unit t = decode_unit(u, p);
-      // Scales and bias of this unit, fetched before its accumulator is ready
-      // (a K split of the weight-row tiling stores raw partial sums and needs
-      // none of them).
-      const bool split = C::WROWS && p.splits > 1;
-      float rscale = 0.0f, rbias = 0.0f;
-      int row_idx;
       if (C::WROWS) {
         const int o = t.m * BM + row_in_tile;
-        row_idx = o;
-        if (o < p.N && !split) {
-          rscale = __ldg(p.s_grp + group_of(o, p.N, p.g));
-          rbias = p.bias ? __half2float(p.bias[o]) : 0.0f;
+        if (o < p.N) {
+          n_rs = __ldg(p.s_grp + group_of(o, p.N, p.g));
+          if (p.bias) n_rb = p.bias[o];
         }
-        for (int c = cb + lane; c < ce && !split; c += 32) {
+#pragma unroll
+        for (int i = 0; i < PCOLS; ++i) {
+          const int c = cb + lane + 32 * i;
           const int tok = t.n * BN + c;
-          colv[c] = tok < p.T ? __ldg(p.s_tok + tok) : 0.0f;
+          if (c < ce && tok < p.T) n_cv[i] = __ldg(p.s_tok + tok);
         }
       } else {
         const int tok = t.m * C::TILE_M + static_cast<int>(crank) * BM + row_in_tile;
-        row_idx = tok;
-        if (tok < p.T) rscale = __ldg(p.s_tok + tok);
-        for (int c = cb + lane; c < ce; c += 32) {
+        if (tok < p.T) n_rs = __ldg(p.s_tok + tok);
+#pragma unroll
+        for (int i = 0; i < PCOLS; ++i) {
+          const int c = cb + lane + 32 * i;
           const int o = t.n * BN + c;
-          colv[c] = o < p.N ? __ldg(p.s_grp + group_of(o, p.N, p.g)) : 0.0f;
-          colb[c] = (o < p.N && p.bias) ? __half2float(p.bias[o]) : 0.0f;
+          if (c < ce && o < p.N) {
+            n_cv[i] = __ldg(p.s_grp + group_of(o, p.N, p.g));
+            if (p.bias) n_cb[i] = p.bias[o];
+          }
         }
       }
+    };
+    fetch(unit0);
+    for (int u = unit0; u < p.num_units; u += ustep) {
+      const Unit t = decode_unit(u, p);
+      const float rscale = n_rs, rbias = __half2float(n_rb);
+#pragma unroll
+      for (int i = 0; i < PCOLS; ++i) {
+        const int c = cb + lane + 32 * i;
+        if (c < ce) {
+          colv[c] = n_cv[i];
+          colb[c] = __half2float(n_cb[i]);
+        }
+      }
+      const int row_idx = C::WROWS ? t.m * BM + row_in_tile
+                                   : t.m * C::TILE_M + static_cast<int>(crank) * BM + row_in_tile;
       __syncwarp();
+      fetch(u + ustep);
       if (!wait_warp(&tfull_bar[buf], tphase, abort_flag, p.status, 4)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
@@ -564,59 +598,63 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
               }
             }
           }
-        } else {
-          // lane = token, columns = output features
-          const int tok = row_idx;
-          const int o0 = t.n * BN + c0;
-          uint32_t h[16];
-          if (tok < p.T && o0 < p.N) {
+        }
+      };
+      // token-row tiling, lane = token, columns = output features: dequantize
+      // 32 accumulator columns into 16 packed fp16 pairs
+      auto dequant_tok = [&](const uint32_t (&acc)[32], int c0, uint32_t (&h)[16]) {
+        const int tok = row_idx;
+        const int o0 = t.n * BN + c0;
+        if (tok < p.T && o0 < p.N) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-              const float4 sv = *reinterpret_cast<const float4*>(colv + c0 + j);
-              const float4 bv = *reinterpret_cast<const float4*>(colb + c0 + j);
-              float v0 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), rscale);
-              float v1 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), rscale);
-              float v2 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 2])), rscale);
-              float v3 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 3])), rscale);
-              v0 = __fadd_rn(__fmul_rn(v0, sv.x), bv.x);
-              v1 = __fadd_rn(__fmul_rn(v1, sv.y), bv.y);
-              v2 = __fadd_rn(__fmul_rn(v2, sv.z), bv.z);
-              v3 = __fadd_rn(__fmul_rn(v3, sv.w), bv.w);
-              h[j / 2] = pack_half2(v0, v1);
-              h[j / 2 + 1] = pack_half2(v2, v3);
-            }
-            int32_t* arow = p.acc_dbg ? p.acc_dbg + static_cast<size_t>(tok) * p.N + o0 : nullptr;
-            if (arow) {
+          for (int j = 0; j < 32; j += 4) {
+            const float4 sv = *reinterpret_cast<const float4*>(colv + c0 + j);
+            const float4 bv = *reinterpret_cast<const float4*>(colb + c0 + j);
+            float v0 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j])), rscale);
+            float v1 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 1])), rscale);
+            float v2 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 2])), rscale);
+            float v3 = __fmul_rn(__int2float_rn(static_cast<int>(acc[j + 3])), rscale);
+            v0 = __fadd_rn(__fmul_rn(v0, sv.x), bv.x);
+            v1 = __fadd_rn(__fmul_rn(v1, sv.y), bv.y);
+            v2 = __fadd_rn(__fmul_rn(v2, sv.z), bv.z);
+            v3 = __fadd_rn(__fmul_rn(v3, sv.w), bv.w);
+            h[j / 2] = pack_half2(v0, v1);
+            h[j / 2 + 1] = pack_half2(v2, v3);
+          }
+          int32_t* arow = p.acc_dbg ? p.acc_dbg + static_cast<size_t>(tok) * p.N + o0 : nullptr;
+          if (arow) {
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                if (o0 + 8 * q < p.N) {  // N % 8 == 0: 8-column chunks are all in or all out
-                  reinterpret_cast<uint4*>(arow)[2 * q] =
-                      make_uint4(acc[8 * q], acc[8 * q + 1], acc[8 * q + 2], acc[8 * q + 3]);
-                  reinterpret_cast<uint4*>(arow)[2 * q + 1] = make_uint4(
-                      acc[8 * q + 4], acc[8 * q + 5], acc[8 * q + 6], acc[8 * q + 7]);
-                }
+            for (int q = 0; q < 4; ++q) {
+              if (o0 + 8 * q < p.N) {  // N % 8 == 0: 8-column chunks are all in or all out
+                reinterpret_cast<uint4*>(arow)[2 * q] =
+                    make_uint4(acc[8 * q], acc[8 * q + 1], acc[8 * q + 2], acc[8 * q + 3]);
+                reinterpret_cast<uint4*>(arow)[2 * q + 1] = make_uint4(
+                    acc[8 * q + 4], acc[8 * q + 5], acc[8 * q + 6], acc[8 * q + 7]);
               }
             }
           }
-          // The warp's 32 rows x 32 columns go out as one TMA tensor store
-          // (rows past T / columns past N are clipped by the TMA unit): wait
-          // until the previous store has read the staging buffer, write this
-          // lane's 64-byte row in the 64B-swizzled layout, then issue.
-          const int row0 = t.m * C::TILE_M + static_cast<int>(crank) * BM + quad * 32;
-          if (o0 < p.N && row0 < p.T) {  // warp-uniform
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
-            const int sw = (lane >> 1) & 3;
+        }
+      };
+      // The warp's 32 rows x 32 columns go out as one TMA tensor store (rows
+      // past T / columns past N are clipped by the TMA unit): wait until the
+      // previous store has read the staging buffer, write this lane's
+      // 64-byte row in the 64B-swizzled layout, then issue.
+      auto store_tok = [&](const uint32_t* h, int c0) {
+        const int o0 = t.n * BN + c0;
+        const int row0 = t.m * C::TILE_M + static_cast<int>(crank) * BM + quad * 32;
+        if (o0 < p.N && row0 < p.T) {  // warp-uniform
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
+          const int sw = (lane >> 1) & 3;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ sw) << 4)) =
-                  make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_2d(&map_y, stg, o0, row0);
-              bulk_commit_group();
-            }
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(stg + lane * 64 + ((q ^ sw) << 4)) =
+                make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_y, stg, o0, row0);
+            bulk_commit_group();
           }
         }
       };
@@ -644,7 +682,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           }
           process(a0, c0);
         }
-      } else {
+      } else if constexpr (C::WROWS) {
       // Two 32-column TMEM loads in flight before each wait.
 #pragma unroll 1
       for (int c0 = cb; c0 < ce; c0 += 64) {
@@ -663,15 +701,48 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         process(a0, c0);
         if (two) process(a1, c0 + 32);
       }
+      } else {
+        // Token rows: dequantize and store 64 columns at a time, then release
+        // the accumulator buffer.  (Dequantizing a warp's whole column range
+        // into registers and releasing the buffer before the stores measured
+        // slower: the stores then run back to back, each waiting for the
+        // previous one to leave the staging buffer.)
+#pragma unroll 1
+        for (int c0 = cb; c0 < ce; c0 += 64) {
+          uint32_t a0[32], a1[32];
+          const bool two = c0 + 32 < ce;
+          tmem_ld_32x32b_x32(t_row + c0, a0);
+          if (two) tmem_ld_32x32b_x32(t_row + c0 + 32, a1);
+          tmem_ld_wait();
+          if (C::W4) {  // INT4 weights were widened as codes*16: exact division
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
+              a1[j] = static_cast<uint32_t>(static_cast<int>(a1[j]) >> 4);
+            }
+          }
+          uint32_t h[16];
+          dequant_tok(a0, c0, h);
+          store_tok(h, c0);
+          if (two) {
+            dequant_tok(a1, c0 + 32, h);
+            store_tok(h, c0 + 32);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (C::PAIR)
+            mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+          else
+            mbar_arrive(&tempty_bar[buf]);
+        }
       }
-      // Release the accumulator buffer to the MMA warp (the leader's, for a pair).
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if constexpr (C::PAIR)
-          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
-        else
-          mbar_arrive(&tempty_bar[buf]);
+      if constexpr (C::WROWS) {
+        // Release the accumulator buffer to the MMA warp.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty_bar[buf]);
       }
       if (++buf == 2) {
         buf = 0;
@@ -854,6 +925,12 @@ struct Plan {
 };
 
 int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// fp16 output [T][N]: 32 x 32 boxes written by the epilogue warps
+bool encode_y_map(CUtensorMap* my, void* Y, int T, int N) {
+  return encode_tma_2d(my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
+                       32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
 
 // Wave-aware cost in MMA cycles: ceil(units/SMs) * k-blocks per unit * 2*BN
 // (a 128 x BN x 128 int8 block takes about 2*BN cycles), plus a fixed
@@ -1083,9 +1160,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
                        CU_TENSOR_MAP_SWIZZLE_128B))
       return ZQ_ERR_CUDA;
   }
-  // fp16 output [T][N]: 32 x 32 boxes written by the epilogue warps
-  if (!encode_tma_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
-                     32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+  if (!encode_y_map(&my, Y, T, N))
     return ZQ_ERR_CUDA;
 
   int grid = std::min(plan.units, sms);
@@ -1231,8 +1306,7 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, BK, w_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return ZQ_ERR_CUDA;
-  if (!encode_tma_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
-                     32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+  if (!encode_y_map(&my, Y, T, N))
     return ZQ_ERR_CUDA;
 
   int grid = std::min(plan.units, sms);

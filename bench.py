@@ -14,7 +14,9 @@ Prints ONE JSON line (rank 0).  `value` is int8 TOPS of the whole step
 (2*T*N*K summed over the four GEMMs / step time) with inputs resident in HBM;
 `e2e` is the same through the C ABI with the step's fp16 inputs copied from
 pinned host memory and its fp16 outputs copied back inside the timed region.
-The L2 is flushed (a 512 MB write) before every timed step.
+The L2 is flushed before every timed step: a 512 MB write, then a 256 MB
+read, so that the timed region starts with a cold L2 holding no dirty lines
+of the flush itself (their write-back would otherwise land inside it).
 """
 from __future__ import annotations
 
@@ -189,8 +191,20 @@ class LayerStep:
             self.run_gemm(it, stream)
 
 
+def make_flush_buffers(device):
+    """A 512 MB buffer that the flush writes and a 256 MB one that it reads
+    (both larger than the 126 MB L2), plus the read's scalar result."""
+    w = torch.zeros(512 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    r = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    return w, r, torch.empty((), dtype=torch.float32, device=device)
+
+
 def flush_l2(buf):
-    buf.add_(1)
+    """Evict the L2: write a buffer larger than it, then read another one so
+    that the lines left behind are clean."""
+    w, r, out = buf
+    w.add_(1)
+    torch.sum(r, dim=0, out=out)
 
 
 def barrier(dist_on):
@@ -245,8 +259,7 @@ def gpu_arm(args, dist_on, rank, world):
     step = LayerStep(zq, inputs, device)
     torch.cuda.synchronize()
     wquant_s = time.perf_counter() - t0
-    flush_buf = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-    flush_buf.zero_()
+    flush_buf = make_flush_buffers(device)
 
     for _ in range(args.warmup):
         step.run()
@@ -281,7 +294,11 @@ def gpu_arm(args, dist_on, rank, world):
     eager_ms /= max(3, args.steps // 2)
 
     # ---- per-kernel device times for the roofline: a CUDA graph of R x
-    # [L2 flush, kernel] minus a graph of R x [L2 flush], divided by R
+    # [L2 flush, kernel] minus a graph of R x [L2 flush], divided by R, both
+    # timed with CUDA events on the launching stream.  (Events between the
+    # launches of an eager step would also count each kernel's launch
+    # latency, which the step's graph with programmatic dependent launch
+    # hides.)
     reps = max(3, min(args.steps, 20))
 
     def graph_of(fn):
@@ -372,7 +389,7 @@ def gpu_arm(args, dist_on, rank, world):
             "workload": f"{layer} layer, T={T} tokens, 4 quantized linears "
                         + ", ".join(f"{s.name} {s.K}->{s.N} W{s.bits}A8 g={s.g}" for s in specs),
             "tokens": T,
-            "l2": "flushed before every timed step (512 MB write)",
+            "l2": "flushed before every timed step (512 MB write, then 256 MB read)",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "launch": "cuda graph replay of the step" if graph is not None else "eager launches",
         },

@@ -34,7 +34,7 @@ def main():
     ap.add_argument("--pair", type=int, default=0, help="1 = single-CTA tiles, 2 = CTA pairs")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
     ap.add_argument("--flush", action="store_true",
-                    help="write a 512 MB buffer before every launch (cold L2, as in bench.py)")
+                    help="flush the L2 before every launch (512 MB write + 256 MB read, as in bench.py)")
     a = ap.parse_args()
 
     T = a.tokens or synth.LAYERS[a.layer].tokens[0]
@@ -50,11 +50,17 @@ def main():
     Y = torch.empty((T, s.N), dtype=torch.float16, device="cuda")
     gemm = zq.gemm_w4a8 if s.bits == 4 else zq.gemm_w8a8
 
-    flush = torch.empty(128 * 1024 * 1024, dtype=torch.float32, device="cuda") if a.flush else None
+    # L2 flush: write 512 MB, then read 256 MB, so the L2 is cold and clean
+    flush = None
+    if a.flush:
+        flush = (torch.zeros(128 * 1024 * 1024, dtype=torch.float32, device="cuda"),
+                 torch.ones(64 * 1024 * 1024, dtype=torch.float32, device="cuda"),
+                 torch.empty((), dtype=torch.float32, device="cuda"))
 
     def run():
         if flush is not None:
-            flush.add_(1)
+            flush[0].add_(1)
+            torch.sum(flush[1], dim=0, out=flush[2])
         if a.kind == "gemm":
             gemm(Xq, st, Wq, sg, b, Y=Y)
         elif a.kind == "ln":

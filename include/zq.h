@@ -102,8 +102,10 @@ zq_status zq_ln_quant(const void* X, const void* gamma, const void* beta, int T,
  *               acc[t][o] = sum_k Xq[t][k]*Wq[o][k]   (exact, int32)
  *               Y[t][o] = fp16(((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]))
  *   acc_dbg     int32 [T][N] or NULL: also store acc (for checking).
- * Runs on tcgen05 tensor cores.  Small T (weight-streaming) shapes split K
- * across SMs: the exact int32 partial sums go to a library-owned workspace
+ * Runs on tcgen05 tensor cores, except for T <= 2 (INT8) or T <= 4 (INT4
+ * weights), a memory-bound matrix-vector product that runs on CUDA cores
+ * (dp4a, exact int32).  Small T (weight-streaming) tensor-core shapes split
+ * K across SMs: the exact int32 partial sums go to a library-owned workspace
  * and a second kernel on the same stream adds them and dequantizes; calls
  * that use the workspace on different streams must not overlap.
  * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
@@ -164,7 +166,10 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  * tests and benchmarks to force one kernel variant.  0 always means
  * "automatic".  Unknown keys return ZQ_ERR_UNSUPPORTED.
  *   ZQ_OPT_GEMM_PATH   1 = token rows on the MMA M side (prefill tiling),
- *                      2 = weight rows on the MMA M side (weight streaming).
+ *                      2 = weight rows on the MMA M side (weight streaming),
+ *                      3 = CUDA-core matrix-vector product (T <= 4, else
+ *                          ZQ_ERR_UNSUPPORTED); automatic at T <= 4 with
+ *                          INT4 weights and at T <= 2 with INT8 ones.
  *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256).
  *   ZQ_OPT_SPLIT_K     number of K splits for path 2 (1 = none).
  *   ZQ_OPT_MAX_CTAS    cap on the number of CTAs of the GEMM (persistent grid).

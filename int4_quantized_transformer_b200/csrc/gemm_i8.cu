@@ -75,16 +75,23 @@ struct Cfg {
   static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // token rows per unit (token-row tiling)
   static constexpr int ACT_ROWS = WROWS ? BN : BM;
   static constexpr int W_ROWS = WROWS ? BM : (PAIR ? BN / 2 : BN);
-  static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * BK;
-  static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) : 0;
   // Weight streaming with INT4 weights: the packed slices (with the small
   // activation tiles) get a deep ring of their own, so that many bytes are
   // in flight from HBM, while the unpacked weights use a shallow ring that
   // only the unpack warps and the MMA cycle through.
-  // In this mode the deep ring holds, per K slice, the packed weights and
-  // the activation tile (B); the shallow ring holds only unpacked weights (A).
+  // In this mode the deep ring holds, per stage, the packed weights and the
+  // activation tiles (B); the shallow ring holds only unpacked weights (A).
   static constexpr bool DEEP = WROWS && W4;
+  // K slices per pipeline stage.  INT4 weight streaming carries two (up to
+  // BN = 128, where two deep slots of two slices still fit), so the
+  // per-stage cost (waits, commits, the unpack handoff) is paid once per
+  // 16 KB of packed weights instead of once per 8 KB.
+  static constexpr int KPS = (DEEP && BN <= 128) ? 2 : 1;
+  static constexpr int A_SLICE = BM * BK;                          // one K slice of A
+  static constexpr int B_SLICE = (PAIR ? BN / 2 : BN) * BK;        // one K slice of B
+  static constexpr int A_BYTES = A_SLICE * KPS;
+  static constexpr int B_BYTES = B_SLICE * KPS;
+  static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) * KPS : 0;  // packed row = KPS * 64 bytes
   // Weight streaming is bound by how fast TMA copies are issued: one issuing
   // thread per SM keeps well under the HBM bandwidth in flight, two do not.
   // The second producer warp is the last warp of the CTA; the producers take
@@ -99,10 +106,11 @@ struct Cfg {
   static constexpr int FREE_BYTES =
       kSmemBudget - NUM_EPI_WARPS_C * STG_BYTES - 8 * EPI_COLS * 8;
   static constexpr int STAGE_BYTES = DEEP ? A_BYTES : A_BYTES + B_BYTES + P_BYTES;
-  static constexpr int STAGES_RAW = DEEP ? 4 : FREE_BYTES / STAGE_BYTES;
+  static constexpr int STAGES_RAW = DEEP ? (KPS == 2 ? 2 : 4) : FREE_BYTES / STAGE_BYTES;
   static constexpr int STAGES_CAP = WROWS ? 12 : 8;
   static constexpr int STAGES_ANY = STAGES_RAW > STAGES_CAP ? STAGES_CAP : STAGES_RAW;
-  static constexpr int STAGES = NUM_PROD_WARPS == 2 ? STAGES_ANY & ~1 : STAGES_ANY;
+  // the producers fill the shallow ring only when there is no deep ring
+  static constexpr int STAGES = (NUM_PROD_WARPS == 2 && !DEEP) ? STAGES_ANY & ~1 : STAGES_ANY;
   static constexpr int PSTAGES_RAW =
       DEEP ? (FREE_BYTES - STAGES * STAGE_BYTES) / (P_BYTES + B_BYTES) : STAGES;
   static constexpr int PSTAGES_ANY = PSTAGES_RAW > 16 ? 16 : PSTAGES_RAW;
@@ -136,7 +144,7 @@ struct Cfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGES >= 2 && PSTAGES >= 2, "not enough shared memory for two stages");
-  static_assert(NUM_PROD_WARPS == 1 || (STAGES % 2 == 0 && (!DEEP || PSTAGES % 2 == 0)),
+  static_assert(NUM_PROD_WARPS == 1 || (DEEP ? PSTAGES % 2 == 0 : STAGES % 2 == 0),
                 "two producers need rings with an even number of slots");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(!PAIR || (BN / 2) % 8 == 0, "B half-tile rows must fill 8-row swizzle atoms");
@@ -174,8 +182,12 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmParams& p) {
   return r;
 }
 
+// group(o) = floor(o * g / N); a 32-bit division whenever o * g fits in 32
+// bits (N * g < 2^32 covers every layer shape), else a 64-bit one.
 __device__ __forceinline__ int group_of(int o, int N, int g) {
-  return static_cast<int>((static_cast<long long>(o) * g) / N);
+  const unsigned long long prod = static_cast<unsigned long long>(o) * static_cast<unsigned>(g);
+  if (prod < (1ull << 32)) return static_cast<int>(static_cast<unsigned>(prod) / static_cast<unsigned>(N));
+  return static_cast<int>(prod / static_cast<unsigned>(N));
 }
 
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast, and
@@ -294,7 +306,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       // the deep ring
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_act = l2_policy_evict_last();
-      constexpr uint32_t bytes = static_cast<uint32_t>(C::P_BYTES + C::ACT_ROWS * BK);
+      constexpr uint32_t bytes = static_cast<uint32_t>(C::P_BYTES + C::B_BYTES);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t fills[16];
@@ -302,7 +314,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ok = true;
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
           if (NP > 1 && (seq++ % NP) != pid) {
             if (++stage == C::PSTAGES) {
               stage = 0;
@@ -315,10 +327,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             break;
           }
           mbar_arrive_expect_tx(&pfull_bar[stage], bytes);
+          // KPS K slices: one packed box KPS*64 bytes wide, KPS activation
+          // tiles (a slice past K reads the TMA's zero fill: it adds nothing)
           tma_load_2d(sP + stage * C::P_BYTES, &map_w, &pfull_bar[stage], kb * (BK / 2), t.m * BM,
                       pol_w);
-          tma_load_2d(sB + stage * C::B_BYTES, &map_act, &pfull_bar[stage], kb * BK, t.n * BN,
-                      pol_act);
+#pragma unroll
+          for (int h = 0; h < C::KPS; ++h)
+            tma_load_2d(sB + stage * C::B_BYTES + h * C::B_SLICE, &map_act, &pfull_bar[stage],
+                        (kb + h) * BK, t.n * BN, pol_act);
           ++fills[stage];
           if (++stage == C::PSTAGES) {
             stage = 0;
@@ -346,7 +362,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         const Unit t = decode_unit(u, p);
         const int act_row = C::WROWS ? t.n * BN : t.m * C::TILE_M + static_cast<int>(crank) * BM;
         const int w_row = C::WROWS ? t.m * BM : t.n * BN + static_cast<int>(crank) * C::W_ROWS;
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
           if (NP > 1 && (seq++ % NP) != pid) {
             if (++stage == STAGES) {
               stage = 0;
@@ -425,7 +441,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, p.status, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::BUF_COLS);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
           uint64_t* rb = C::W4 ? &ready_bar[stage] : &full_bar[stage];
           if (!mbar_wait(rb, phase, abort_flag, p.status, 3)) {
             ok = false;
@@ -443,19 +459,23 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES));
-          const uint64_t db =
-              make_sw128_desc(smem_u32(sB + (C::DEEP ? pst : stage) * C::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            // advance the start address by k*32 bytes (>>4 = 2k) inside the swizzle row
-            if constexpr (C::PAIR)
-              mma_i8_pair(d_tmem, da + static_cast<uint64_t>(2 * k),
-                          db + static_cast<uint64_t>(2 * k), idesc, (kb > t.kb0 || k > 0) ? 1u : 0u);
-            else
-              mma_i8(d_tmem + static_cast<uint32_t>((k % C::NACC) * C::ACC_STRIDE),
-                     da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), idesc,
-                     (kb > t.kb0 || k >= C::NACC) ? 1u : 0u);
+          for (int h = 0; h < C::KPS; ++h) {
+            const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES + h * C::A_SLICE));
+            const uint64_t db = make_sw128_desc(
+                smem_u32(sB + (C::DEEP ? pst : stage) * C::B_BYTES + h * C::B_SLICE));
+            const bool first = kb == t.kb0 && h == 0;  // the unit's first K slice
+#pragma unroll
+            for (int k = 0; k < BK / UMMA_K; ++k) {
+              // advance the start address by k*32 bytes (>>4 = 2k) inside the swizzle row
+              if constexpr (C::PAIR)
+                mma_i8_pair(d_tmem, da + static_cast<uint64_t>(2 * k),
+                            db + static_cast<uint64_t>(2 * k), idesc, (!first || k > 0) ? 1u : 0u);
+              else
+                mma_i8(d_tmem + static_cast<uint32_t>((k % C::NACC) * C::ACC_STRIDE),
+                       da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), idesc,
+                       (!first || k >= C::NACC) ? 1u : 0u);
+            }
           }
           if constexpr (C::PAIR)
             mma_commit_pair_mc(&empty_bar[stage], 0x3);
@@ -570,9 +590,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       const int row_idx = C::WROWS ? t.m * BM + row_in_tile
                                    : t.m * C::TILE_M + static_cast<int>(crank) * BM + row_in_tile;
       __syncwarp();
-      fetch(u + ustep);
       if (!wait_warp(&tfull_bar[buf], tphase, abort_flag, p.status, 4)) break;
       tc_fence_after();
+      // the next unit's loads are in flight while this unit is processed
+      fetch(u + ustep);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(buf * C::BUF_COLS);
 
@@ -756,7 +777,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       const int ut = threadIdx.x - 32 * (2 + C::NUM_EPI_WARPS);  // 0 .. 32*NUM_UNPACK_WARPS-1
       constexpr int UROWS = 4 * C::NUM_UNPACK_WARPS;  // rows of one unpack step
       const int ur = ut >> 3, uj = ut & 7;
-      const int unp_src = ur * (BK / 2) + uj * 8;
+      constexpr int PROW = (BK / 2) * C::KPS;  // bytes of one packed row in a stage
+      const int unp_src = ur * PROW + uj * 8;
       const int unp_dst = ur * BK + ((uj ^ (ur & 7)) << 4);
       int stage = 0;
       uint32_t phase = 0;
@@ -765,7 +787,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ok = true;
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
           if constexpr (C::DEEP) {
             // the packed slice has landed, and the MMA has released the slot
             // of the shallow ring that the unpacked weights go to
@@ -783,15 +805,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           // r = ut / 8 + UROWS i: stepping a multiple of 8 rows keeps r % 8,
           // hence the swizzled chunk position, fixed, so the shared-memory
           // offsets are per-thread constants plus i * (UROWS rows).
-          const uint8_t* src = sP + (C::DEEP ? pst : stage) * C::P_BYTES + unp_src;
-          uint8_t* dst = (C::WROWS ? sA + stage * C::A_BYTES : sB + stage * C::B_BYTES) + unp_dst;
 #pragma unroll
-          for (int i = 0; i < C::W_ROWS / UROWS; ++i) {
-            const uint2 pk = *reinterpret_cast<const uint2*>(src + i * UROWS * (BK / 2));
-            uint4 o;
-            unpack8_x16(pk.x, o.x, o.y);
-            unpack8_x16(pk.y, o.z, o.w);
-            *reinterpret_cast<uint4*>(dst + i * UROWS * BK) = o;
+          for (int h = 0; h < C::KPS; ++h) {
+            const uint8_t* src = sP + (C::DEEP ? pst : stage) * C::P_BYTES + unp_src + h * (BK / 2);
+            uint8_t* dst = (C::WROWS ? sA + stage * C::A_BYTES + h * C::A_SLICE
+                                     : sB + stage * C::B_BYTES + h * C::B_SLICE) +
+                           unp_dst;
+#pragma unroll
+            for (int i = 0; i < C::W_ROWS / UROWS; ++i) {
+              const uint2 pk = *reinterpret_cast<const uint2*>(src + i * UROWS * PROW);
+              uint4 o;
+              unpack8_x16(pk.x, o.x, o.y);
+              unpack8_x16(pk.y, o.z, o.w);
+              *reinterpret_cast<uint4*>(dst + i * UROWS * BK) = o;
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -921,10 +948,14 @@ struct Plan {
   bool pair;
   int bn;
   int m_tiles, n_tiles, k_blocks, splits, kb_per_split, units;
+  int kps = 1;  // K slices per pipeline stage (weight rows with INT4 weights: 2)
   double cost;
 };
 
 int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Largest token count the automatic choice sends to the matrix-vector path.
+int gemv_max_tokens(bool w4) { return w4 ? kGemvMaxTokens : 2; }
 
 // fp16 output [T][N]: 32 x 32 boxes written by the epilogue warps
 bool encode_y_map(CUtensorMap* my, void* Y, int T, int N) {
@@ -935,34 +966,39 @@ bool encode_y_map(CUtensorMap* my, void* Y, int T, int N) {
 // Wave-aware cost in MMA cycles: ceil(units/SMs) * k-blocks per unit * 2*BN
 // (a 128 x BN x 128 int8 block takes about 2*BN cycles), plus a fixed
 // charge per extra wave and per split-K reduction.
-Plan plan_wrows(int T, int N, int K, int sms, int forced_split) {
+// K is split in whole stages of kps K slices: two for INT4 weights up to
+// BN = 128 (Cfg::KPS), else one.
+Plan plan_wrows(int T, int N, int K, int sms, int forced_split, bool w4) {
   Plan p{};
   p.wrows = true;
   p.pair = false;
   int bn = 16;
   while (bn < T && bn < 256) bn *= 2;
   p.bn = bn;
+  const int kps = (w4 && bn <= 128) ? 2 : 1;
+  p.kps = kps;
   p.m_tiles = ceil_div(N, BM);
   p.n_tiles = ceil_div(T, bn);
   p.k_blocks = ceil_div(K, BK);
   const int tiles = p.m_tiles * p.n_tiles;
+  const int k_stages = ceil_div(p.k_blocks, kps);
   double best = 1e30;
   int best_s = 1;
-  const int max_s = forced_split > 0 ? forced_split : std::min(p.k_blocks, 32);
-  const int min_s = forced_split > 0 ? forced_split : 1;
+  const int max_s = forced_split > 0 ? std::min(forced_split, k_stages) : std::min(k_stages, 32);
+  const int min_s = forced_split > 0 ? max_s : 1;
   for (int s = min_s; s <= max_s; ++s) {
-    const int kbps = ceil_div(p.k_blocks, s);
-    const int s_eff = ceil_div(p.k_blocks, kbps);
+    const int sps = ceil_div(k_stages, s);  // stages per split
+    const int s_eff = ceil_div(k_stages, sps);
     const int units = tiles * s_eff;
     const int waves = ceil_div(units, sms);
     // the unit time is set by streaming its weights (HBM-bound): count bytes
-    const double cost = waves * (kbps * 1.0 + 2.0) + (s_eff > 1 ? 1.0 : 0.0);
+    const double cost = waves * (sps * kps + 2.0) + (s_eff > 1 ? 1.0 : 0.0);
     if (cost < best - 1e-9) {
       best = cost;
       best_s = s_eff;
     }
   }
-  p.kb_per_split = ceil_div(p.k_blocks, best_s);
+  p.kb_per_split = kps * ceil_div(k_stages, best_s);
   p.splits = ceil_div(p.k_blocks, p.kb_per_split);
   p.units = tiles * p.splits;
   p.cost = best * 2.0 * 256;  // comparable scale with the token-row plan
@@ -1088,12 +1124,22 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int sms = num_sms();
 
-  // Weight rows on the MMA M side for small token counts (weight streaming),
-  // token rows otherwise; tests and benchmarks may force either.
+  // A handful of tokens: the CUDA-core matrix-vector path (measured faster
+  // than the tensor-core tilings up to T = 4 with INT4 weights and up to
+  // T = 2 with INT8 ones).  Otherwise weight rows on the MMA M side for small
+  // token counts (weight streaming), token rows beyond; tests and benchmarks
+  // may force any of them.
   const int forced_path = option(ZQ_OPT_GEMM_PATH);
+  if (forced_path == 3 || (forced_path == 0 && T <= gemv_max_tokens(w4))) {
+    if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
+    return launch_gemv_i8(w4 ? 4 : 8, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg,
+                          option(ZQ_OPT_MAX_CTAS), st) == cudaSuccess
+               ? ZQ_OK
+               : ZQ_ERR_CUDA;
+  }
   Plan plan;
   if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
-    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K));
+    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K), w4);
   } else {
     const int fbn = option(ZQ_OPT_GEMM_BN);
     if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
@@ -1152,8 +1198,9 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return ZQ_ERR_CUDA;
   if (w4) {
-    if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K / 2, N, K / 2, BK / 2, w_rows,
-                       CU_TENSOR_MAP_SWIZZLE_NONE))
+    // one box per stage: plan.kps K slices of 64 packed bytes per row
+    if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K / 2, N, K / 2,
+                       plan.kps * (BK / 2), w_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
       return ZQ_ERR_CUDA;
   } else {
     if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, BK, w_rows,
@@ -1259,9 +1306,17 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   const int sms = num_sms();
 
   const int forced_path = option(ZQ_OPT_GEMM_PATH);
+  // the matrix-vector path (as in zq_gemm_w8a8) needs no scratch at all
+  if (forced_path == 3 || (forced_path == 0 && T <= gemv_max_tokens(false))) {
+    if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
+    return launch_gemv_i8(8, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg,
+                          option(ZQ_OPT_MAX_CTAS), st) == cudaSuccess
+               ? ZQ_OK
+               : ZQ_ERR_CUDA;
+  }
   Plan plan;
   if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
-    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K));
+    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K), false);
   } else {
     const int fbn = option(ZQ_OPT_GEMM_BN);
     if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;

@@ -19,6 +19,13 @@ constexpr int kDevErrTimeoutBase = 1000;
 // Device pointer of the current device's status word (set up once per device).
 int* device_status_ptr();
 int num_sms();
+
+// The CUDA-core matrix-vector path of the quantized linear layer, for at most
+// kGemvMaxTokens tokens (gemv_i8.cu): bits = 4 (packed INT4) or 8.
+constexpr int kGemvMaxTokens = 4;
+cudaError_t launch_gemv_i8(int bits, const int8_t* Xq, const float* s_tok, const void* W,
+                           const float* s_grp, int g, const void* bias, int T, int N, int K,
+                           void* Y, int32_t* acc_dbg, int max_ctas, cudaStream_t st);
 int option(int key);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.

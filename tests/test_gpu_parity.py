@@ -249,6 +249,48 @@ def test_gemm_zero_scales_give_bias(zq):
     assert_bits_equal(Y, np.broadcast_to(b, (T, N)))
 
 
+# ------------------------------------------------------------ matrix-vector path (T <= 4)
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+@pytest.mark.parametrize("N,K,g", [(256, 64, 4), (1000, 4160, 5), (8, 96, 1), (4104, 3072, 24)])
+def test_gemv_path(zq, bits, T, N, K, g):
+    """The CUDA-core matrix-vector path: weight rows go in pairs per warp
+    (the pairs do not fill the last round of warps), K is not a multiple of
+    one round of 32 lanes x 3 chunks, a single group, and T = 3 runs in the
+    four-token kernel."""
+    if bits == 4 and K % 32:
+        pytest.skip("int4 needs K % 32 == 0")
+    _check_gemm(zq, T, N, K, g, bits, seed=T * 7 + N + K, path=3)
+
+
+def test_gemv_persistent_rows_and_extremes(zq):
+    # fewer CTAs than row pairs: every warp walks several pairs
+    _check_gemm(zq, 3, 2048, 1024, 8, 8, seed=21, path=3, max_ctas=3)
+    _check_gemm(zq, 4, 2048, 1024, 8, 4, seed=22, path=3, max_ctas=2)
+    # saturated operands: accumulators reach +-127*127*K (int8) and the INT4
+    # widening multiplies them by 16 before the exact division
+    T, N, K = 4, 64, 8192
+    xq = np.full((T, K), 127, np.int8)
+    xq[1::2] = -127
+    st = np.linspace(1e-3, 1e-2, T).astype(np.float32)
+    sg = np.array([1e-4, 2e-4], np.float32)
+    for bits in (8, 4):
+        w = np.full((N, K), 127 if bits == 8 else 7, np.int8)
+        w[::3] = -127 if bits == 8 else -8
+        Y, acc = _run_gemm(zq, xq, st, w, sg, None, bits, path=3)
+        acc_ref = oracle.gemm_i32(xq, w)
+        assert_bits_equal(acc, acc_ref)
+        assert_fp16_close(Y, oracle.dequant(acc_ref, st, sg, None))
+
+
+def test_gemv_path_rejects_more_tokens(zq):
+    xq, st, wq, sg, b = _quant_operands(5, 64, 64, 2, 8, 1)
+    with pytest.raises(zq.ZQError) as e:
+        _run_gemm(zq, xq, st, wq, sg, b, 8, path=3)
+    assert e.value.status == zq.ZQ_ERR_UNSUPPORTED
+
+
 def test_repeated_split_k_calls_leave_workspace_clean(zq):
     # the split-K workspace must return to zero after every call
     for i in range(3):

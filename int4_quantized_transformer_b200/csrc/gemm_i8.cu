@@ -119,13 +119,7 @@ struct Cfg {
   // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
   // 32-column loads never leave the allocation.
   static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
-  // With weight rows on M the tokens are few (N = BN is small), so one
-  // tcgen05.mma is short and successive MMAs into one accumulator form a
-  // dependent chain whose latency, not the data, sets the pace.  The K steps
-  // of a slice rotate over NACC independent accumulators instead; the
-  // epilogue adds them (exact int32 sums).
-  static constexpr int NACC = WROWS ? (BN <= 64 ? 4 : (BN <= 128 ? 2 : 1)) : 1;
-  static constexpr int BUF_COLS = NACC * ACC_STRIDE;  // TMEM columns per accumulator buffer
+  static constexpr int BUF_COLS = ACC_STRIDE;  // TMEM columns per accumulator buffer
   static constexpr int TMEM_COLS = pow2_at_least(2 * BUF_COLS);
   static constexpr int NUM_EPI_WARPS = NUM_EPI_WARPS_C;
   static constexpr int NUM_UNPACK_WARPS = W4 ? 4 : 0;
@@ -151,7 +145,7 @@ struct Cfg {
   static_assert(!W4 || (W_ROWS % (4 * NUM_UNPACK_WARPS) == 0 && (4 * NUM_UNPACK_WARPS) % 8 == 0),
                 "unpack steps keep the row's swizzle phase");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-  static_assert(TMEM_COLS <= 512 && (BK / UMMA_K) % NACC == 0, "TMEM accumulators");
+  static_assert(TMEM_COLS <= 512, "TMEM accumulators");
   static_assert(EPI_COLS <= 128, "epilogue prefetch holds at most four columns per lane");
 };
 
@@ -472,9 +466,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
                 mma_i8_pair(d_tmem, da + static_cast<uint64_t>(2 * k),
                             db + static_cast<uint64_t>(2 * k), idesc, (!first || k > 0) ? 1u : 0u);
               else
-                mma_i8(d_tmem + static_cast<uint32_t>((k % C::NACC) * C::ACC_STRIDE),
-                       da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k), idesc,
-                       (!first || k >= C::NACC) ? 1u : 0u);
+                mma_i8(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
+                       idesc, (!first || k > 0) ? 1u : 0u);
             }
           }
           if constexpr (C::PAIR)
@@ -680,48 +673,25 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         }
       };
 
-      if constexpr (C::NACC > 1) {
-        // 32 columns at a time: the NACC partial accumulators, added
+      if constexpr (C::WROWS) {
+        // Two 32-column TMEM loads in flight before each wait.
 #pragma unroll 1
-        for (int c0 = cb; c0 < ce; c0 += 32) {
-          uint32_t a0[32], b0[32];
+        for (int c0 = cb; c0 < ce; c0 += 64) {
+          uint32_t a0[32], a1[32];
+          const bool two = c0 + 32 < ce;
           tmem_ld_32x32b_x32(t_row + c0, a0);
-          tmem_ld_32x32b_x32(t_row + C::ACC_STRIDE + c0, b0);
+          if (two) tmem_ld_32x32b_x32(t_row + c0 + 32, a1);
           tmem_ld_wait();
+          if (C::W4) {  // INT4 weights were widened as codes*16: exact division
 #pragma unroll
-          for (int j = 0; j < 32; ++j) a0[j] += b0[j];
-#pragma unroll 1
-          for (int a = 2; a < C::NACC; ++a) {
-            tmem_ld_32x32b_x32(t_row + a * C::ACC_STRIDE + c0, b0);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) a0[j] += b0[j];
-          }
-          if (C::W4) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
+            for (int j = 0; j < 32; ++j) {
+              a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
+              a1[j] = static_cast<uint32_t>(static_cast<int>(a1[j]) >> 4);
+            }
           }
           process(a0, c0);
+          if (two) process(a1, c0 + 32);
         }
-      } else if constexpr (C::WROWS) {
-      // Two 32-column TMEM loads in flight before each wait.
-#pragma unroll 1
-      for (int c0 = cb; c0 < ce; c0 += 64) {
-        uint32_t a0[32], a1[32];
-        const bool two = c0 + 32 < ce;
-        tmem_ld_32x32b_x32(t_row + c0, a0);
-        if (two) tmem_ld_32x32b_x32(t_row + c0 + 32, a1);
-        tmem_ld_wait();
-        if (C::W4) {  // INT4 weights were widened as codes*16: exact division
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
-            a1[j] = static_cast<uint32_t>(static_cast<int>(a1[j]) >> 4);
-          }
-        }
-        process(a0, c0);
-        if (two) process(a1, c0 + 32);
-      }
       } else {
         // Token rows: dequantize and store 64 columns at a time, then release
         // the accumulator buffer.  (Dequantizing a warp's whole column range

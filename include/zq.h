@@ -92,6 +92,30 @@ zq_status zq_ln_quant(const void* X, const void* gamma, const void* beta, int T,
                       int8_t* Xq, float* s_tok, void* Y_ln, zq_stream_t stream);
 
 /*
+ * zq_bias_act_quant -- token-wise dynamic INT8 quantization fused into a
+ * bias-add or a GeLU (Sec. 3.4 "Kernel fusion for token-wise activation
+ * quantization": the quantization is fused with the preceding LayerNorm,
+ * GeLU or bias-add, so the fp16 activation never makes a DRAM round trip).
+ *   X      fp16 [T][K] input rows (tokens), e.g. a GEMM's fp16 output.
+ *   bias   fp16 [K] or NULL (no add).
+ *   act    ZQ_ACT_NONE: v = f32(x) + f32(bias) (one fp32 add), y = fp16(v);
+ *          ZQ_ACT_GELU: y = fp16(gelu(v)), GeLU in its exact form
+ *          gelu(v) = 0.5 v (1 + erf(v / sqrt 2)) = v * 0.5 erfc(-v / sqrt 2),
+ *          evaluated in fp32 with a Chebyshev approximation of erfc
+ *          (fractional error below 1.2e-7; y may differ from a correctly
+ *          rounded GeLU by one fp16 ulp).
+ *   Xq, s_tok  the token quantization of y, as in zq_ln_quant:
+ *          s_tok[t] = amax_t/127 with amax_t = max_k |y|,
+ *          Xq = clamp(rne(y * (127/amax_t)), -127, 127); zero rows give 0.
+ *   Y_act  fp16 [T][K] or NULL: also store y.
+ * Requirements: as zq_ln_quant; act is ZQ_ACT_NONE or ZQ_ACT_GELU
+ * (else ZQ_ERR_UNSUPPORTED).
+ */
+typedef enum { ZQ_ACT_NONE = 0, ZQ_ACT_GELU = 1 } zq_act;
+zq_status zq_bias_act_quant(const void* X, const void* bias, int T, int K, int act, int8_t* Xq,
+                            float* s_tok, void* Y_act, zq_stream_t stream);
+
+/*
  * zq_gemm_w8a8 -- INT8 x INT8 GEMM with the dequantization fused into the
  * epilogue (Sec. 3.4 "CUTLASS INT8 GEMM" and "Dequantization fused into the
  * GEMM epilogue"; Fig. 2 right, second box).

@@ -58,6 +58,36 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 
 // --------------------------------------------------------------- ln_quant
 
+// erfc(a) for a >= 0 in fp32: the Chebyshev approximation of Press, Teukolsky,
+// Vetterling and Flannery, "Numerical Recipes", Sec. 6.2 (erfc with
+// fractional error below 1.2e-7 everywhere), as
+//   erfc(a) ~ t * exp(-a^2 + P(t)),  t = 1 / (1 + a/2),
+// P a degree-9 polynomial, with the hardware exp2.  Fractional (not absolute)
+// accuracy matters here: for negative v, GeLU is v times a tiny erfc.
+__device__ __forceinline__ float erfc_nonneg(float a) {
+  const float t = __frcp_rn(__fmaf_rn(0.5f, a, 1.0f));
+  float p = 0.17087277f;
+  p = __fmaf_rn(p, t, -0.82215223f);
+  p = __fmaf_rn(p, t, 1.48851587f);
+  p = __fmaf_rn(p, t, -1.13520398f);
+  p = __fmaf_rn(p, t, 0.27886807f);
+  p = __fmaf_rn(p, t, -0.18628806f);
+  p = __fmaf_rn(p, t, 0.09678418f);
+  p = __fmaf_rn(p, t, 0.37409196f);
+  p = __fmaf_rn(p, t, 1.00002368f);
+  p = __fmaf_rn(p, t, -1.26551223f);
+  return t * __expf(__fmaf_rn(-a, a, p));
+}
+
+// GeLU, exact form: v * Phi(v) with Phi(v) = 0.5 erfc(-v / sqrt 2), i.e.
+// 0.5 erfc(|v|/sqrt 2) for v <= 0 and 1 - 0.5 erfc(v/sqrt 2) for v > 0 (no
+// cancellation for negative v).  The result stays well within an fp16 ulp of
+// the correctly rounded value; the tests hold it to one fp16 ulp.
+__device__ __forceinline__ float gelu_erf(float v) {
+  const float h = 0.5f * erfc_nonneg(fabsf(v) * 0.70710678118654752f);
+  return v * (v > 0.0f ? 1.0f - h : h);
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -121,9 +151,9 @@ __device__ __forceinline__ float row_tree_sum(float (&cs)[VPT], float* red, int 
 template <int W, int VPT>
 __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 32) : 8) / 2)
     ln_quant_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
-                    const __half* __restrict__ beta, int T, int K, float eps,
-                    int8_t* __restrict__ Xq, float* __restrict__ s_tok,
-                    __half* __restrict__ Y_ln) {
+                    const __half* __restrict__ beta, const __half* __restrict__ act_bias,
+                    int act, int T, int K, float eps, int8_t* __restrict__ Xq,
+                    float* __restrict__ s_tok, __half* __restrict__ Y_ln) {
   constexpr int RT = 32 * W;                // threads per row
   constexpr int RPB = W >= 8 ? 1 : 8 / W;   // rows per block
   constexpr int NBLK = W * (VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4));
@@ -153,6 +183,36 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
       int v = j + i * RT;
       x4[i] = make_uint4(0, 0, 0, 0);
       if (valid && v < nvec) x4[i] = __ldcs(reinterpret_cast<const uint4*>(xr) + v);
+    }
+
+    if (act >= 0) {
+      // the producer of the activation, fused: bias-add (act = 0) or
+      // GeLU (act = 1) of v = f32(x) + f32(bias), rounded to fp16 (the
+      // bias-add is skipped when there is no bias, so x stays bit-exact)
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int v = j + i * RT;
+        if (v < nvec) {
+          const uint4 b4 = act_bias ? __ldg(reinterpret_cast<const uint4*>(act_bias) + v)
+                                    : make_uint4(0, 0, 0, 0);
+          __half2* h = reinterpret_cast<__half2*>(&x4[i]);
+          const __half2* bh = reinterpret_cast<const __half2*>(&b4);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __half22float2(h[e]);
+            if (act_bias) {
+              const float2 bf = __half22float2(bh[e]);
+              f.x = __fadd_rn(f.x, bf.x);
+              f.y = __fadd_rn(f.y, bf.y);
+            }
+            if (act == 1) {
+              f.x = gelu_erf(f.x);
+              f.y = gelu_erf(f.y);
+            }
+            h[e] = __floats2half2_rn(f.x, f.y);
+          }
+        }
+      }
     }
 
     if (ln) {
@@ -260,8 +320,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
 }
 
 template <int W, int VPT>
-cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, int T, int K, float eps,
-                      int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
+cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, const __half* ab, int act,
+                      int T, int K, float eps, int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
   constexpr int RPB = W >= 8 ? 1 : 8 / W;
   constexpr int threads = RPB * 32 * W;
   int per_sm = 0;
@@ -272,20 +332,40 @@ cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, int T, 
   int need = (T + RPB - 1) / RPB;
   int grid = num_sms() * per_sm;
   if (grid > need) grid = need;
-  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, T, K, eps,
-                 Xq, s, Y);
+  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, ab, act, T,
+                 K, eps, Xq, s, Y);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int W>
-cudaError_t launch_ln_w(int vpt, const __half* X, const __half* g, const __half* b, int T, int K,
-                        float eps, int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
+cudaError_t launch_ln_w(int vpt, const __half* X, const __half* g, const __half* b,
+                        const __half* ab, int act, int T, int K, float eps, int8_t* Xq, float* s,
+                        __half* Y, cudaStream_t st) {
   switch (vpt) {
-    case 1: return launch_ln<W, 1>(X, g, b, T, K, eps, Xq, s, Y, st);
-    case 2: return launch_ln<W, 2>(X, g, b, T, K, eps, Xq, s, Y, st);
-    case 3: return launch_ln<W, 3>(X, g, b, T, K, eps, Xq, s, Y, st);
-    default: return launch_ln<W, 4>(X, g, b, T, K, eps, Xq, s, Y, st);
+    case 1: return launch_ln<W, 1>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
+    case 2: return launch_ln<W, 2>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
+    case 3: return launch_ln<W, 3>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
+    default: return launch_ln<W, 4>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
+  }
+}
+
+// Warps per row so that each thread keeps at most 4 vectors of 8 halves;
+// act < 0 selects the LayerNorm (gamma non-NULL) or quant-only form.
+cudaError_t launch_row_quant(const __half* xg, const __half* gg, const __half* bg,
+                             const __half* ab, int act, int T, int K, float eps, int8_t* Xq,
+                             float* s_tok, __half* yg, cudaStream_t st) {
+  const int nvec = K / 8;
+  int W = 1;
+  while (W < 32 && 32 * W * 4 < nvec) W *= 2;
+  const int vpt = (nvec + 32 * W - 1) / (32 * W);
+  switch (W) {
+    case 1: return launch_ln_w<1>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
+    case 2: return launch_ln_w<2>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
+    case 4: return launch_ln_w<4>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
+    case 8: return launch_ln_w<8>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
+    case 16: return launch_ln_w<16>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
+    default: return launch_ln_w<32>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
   }
 }
 
@@ -368,20 +448,23 @@ extern "C" zq_status zq_ln_quant(const void* X, const void* gamma, const void* b
   const __half* bg = gamma ? static_cast<const __half*>(beta) : nullptr;
   __half* yg = static_cast<__half*>(Y_ln);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // warps per row so that each thread keeps at most 4 vectors of 8 halves
-  const int nvec = K / 8;
-  int W = 1;
-  while (W < 32 && 32 * W * 4 < nvec) W *= 2;
-  const int vpt = (nvec + 32 * W - 1) / (32 * W);
-  cudaError_t e;
-  switch (W) {
-    case 1: e = launch_ln_w<1>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st); break;
-    case 2: e = launch_ln_w<2>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st); break;
-    case 4: e = launch_ln_w<4>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st); break;
-    case 8: e = launch_ln_w<8>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st); break;
-    case 16: e = launch_ln_w<16>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st); break;
-    default: e = launch_ln_w<32>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st); break;
-  }
+  const cudaError_t e = launch_row_quant(xg, gg, bg, nullptr, -1, T, K, eps, Xq, s_tok, yg, st);
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+extern "C" zq_status zq_bias_act_quant(const void* X, const void* bias, int T, int K, int act,
+                                       int8_t* Xq, float* s_tok, void* Y_act,
+                                       zq_stream_t stream) {
+  if (act != ZQ_ACT_NONE && act != ZQ_ACT_GELU) return ZQ_ERR_UNSUPPORTED;
+  if (T < 0 || K < 16 || K > 32768 || K % 16 != 0) return ZQ_ERR_SHAPE;
+  if (T == 0) return ZQ_OK;
+  if (!X || !Xq || !s_tok) return ZQ_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq) || (bias && !aligned16(bias)) ||
+      (Y_act && !aligned16(Y_act)))
+    return ZQ_ERR_ALIGN;
+  const cudaError_t e = launch_row_quant(
+      static_cast<const __half*>(X), nullptr, nullptr, static_cast<const __half*>(bias), act, T,
+      K, 0.0f, Xq, s_tok, static_cast<__half*>(Y_act), reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 

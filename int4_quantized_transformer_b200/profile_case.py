@@ -2,6 +2,7 @@
 
     python -m int4_quantized_transformer_b200.profile_case --kind gemm --layer bert_base --gemm 0
     python -m int4_quantized_transformer_b200.profile_case --kind ln --layer bert_base --gemm 0
+    python -m int4_quantized_transformer_b200.profile_case --kind act --act gelu --layer bert_base --gemm 3
 
 Quantizes the weights, runs `--warmup` untimed launches and then `--reps`
 launches of the chosen kernel (the fused LN+quant of that GEMM's input, or
@@ -22,7 +23,9 @@ from int4_quantized_transformer_b200 import synth, zq
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", choices=["gemm", "ln", "wquant"], default="gemm")
+    ap.add_argument("--kind", choices=["gemm", "ln", "act", "wquant"], default="gemm")
+    ap.add_argument("--act", choices=["gelu", "none"], default="gelu",
+                    help="--kind act: GeLU + quant, or bias-add + quant (with a bias)")
     ap.add_argument("--layer", default="bert_base", choices=sorted(synth.LAYERS))
     ap.add_argument("--gemm", type=int, default=0, help="index of the layer's GEMM (0..3)")
     ap.add_argument("--tokens", type=int, default=0)
@@ -47,6 +50,8 @@ def main():
     beta = None if gi.beta is None else gi.beta.cuda()
     Xq, st = zq.ln_quant(X, gamma, beta)
     b = gi.b.cuda()
+    # the bias of the bias-add + quant form: the GEMM's input width
+    act_bias = None if a.act == "gelu" else gi.X[0].cuda() * 0.25
     Y = torch.empty((T, s.N), dtype=torch.float16, device="cuda")
     gemm = zq.gemm_w4a8 if s.bits == 4 else zq.gemm_w8a8
 
@@ -65,6 +70,9 @@ def main():
             gemm(Xq, st, Wq, sg, b, Y=Y)
         elif a.kind == "ln":
             zq.ln_quant(X, gamma, beta, Xq=Xq, s_tok=st)
+        elif a.kind == "act":
+            zq.bias_act_quant(X, act_bias, zq.ACT_GELU if a.act == "gelu" else zq.ACT_NONE,
+                              Xq=Xq, s_tok=st)
         else:
             zq.quantize_weights_groupwise(W, s.g, s.bits, Wq=Wq, s_grp=sg)
 
@@ -96,8 +104,13 @@ def main():
         raise SystemExit(f"device status {rc} ({detail})")
     us = e0.elapsed_time(e1) * 1e3 / a.reps
     ops = 2.0 * T * s.N * s.K
-    print(json.dumps({"kind": a.kind, "layer": a.layer, "gemm": s.name, "T": T, "N": s.N, "K": s.K,
-                      "bits": s.bits, "us": round(us, 2), "tops": round(ops / us / 1e6, 1)}))
+    res = {"kind": a.kind, "layer": a.layer, "gemm": s.name, "T": T, "N": s.N, "K": s.K,
+           "bits": s.bits, "us": round(us, 2)}
+    if a.kind in ("ln", "act"):  # fp16 in, int8 + one fp32 scale per row out
+        res["gbs"] = round((3 * T * s.K + 4 * T) / us / 1e3, 1)
+    else:
+        res["tops"] = round(ops / us / 1e6, 1)
+    print(json.dumps(res))
 
 
 if __name__ == "__main__":

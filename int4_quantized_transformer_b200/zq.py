@@ -23,7 +23,7 @@ OPT_GEMM_PATH, OPT_GEMM_BN, OPT_SPLIT_K, OPT_MAX_CTAS, OPT_CTA_PAIR = 1, 2, 3, 4
 EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
-    "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc",
+    "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant",
 )
 
 
@@ -51,6 +51,7 @@ def _load():
         "zq_get_option": ([I], I),
         "zq_debug_wait_timeout": ([P], I),
         "zq_gemm_w8a8_noalloc": ([P, P, P, P, I, P, I, I, I, P, P, P], I),
+        "zq_bias_act_quant": ([P, P, I, I, I, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -163,6 +164,26 @@ def ln_quant(X: torch.Tensor, gamma=None, beta=None, eps: float = 1e-5, Xq=None,
         _dev(beta, torch.float16, (K,), "beta"), T, K, float(eps),
         _dev(Xq, torch.int8, (T, K), "Xq"), _dev(s_tok, torch.float32, (T,), "s_tok"),
         _dev(y_ln, torch.float16, (T, K), "Y_ln"), _stream(stream)), "zq_ln_quant")
+    return Xq, s_tok
+
+
+ACT_NONE, ACT_GELU = 0, 1
+
+
+def bias_act_quant(X: torch.Tensor, bias=None, act: int = ACT_NONE, Xq=None, s_tok=None, y=None,
+                   stream=None):
+    """Token-wise INT8 quantization fused into a bias-add (act=ACT_NONE) or a
+    GeLU (act=ACT_GELU) (zq_bias_act_quant).  Returns (Xq int8 [T,K],
+    s_tok fp32 [T]); y, if given, receives the fp16 activation."""
+    T, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
+    if s_tok is None:
+        s_tok = torch.empty(T, dtype=torch.float32, device=X.device)
+    _check(_lib.zq_bias_act_quant(
+        _dev(X, torch.float16, (T, K), "X"), _dev(bias, torch.float16, (K,), "bias"), T, K,
+        int(act), _dev(Xq, torch.int8, (T, K), "Xq"), _dev(s_tok, torch.float32, (T,), "s_tok"),
+        _dev(y, torch.float16, (T, K), "Y_act"), _stream(stream)), "zq_bias_act_quant")
     return Xq, s_tok
 
 

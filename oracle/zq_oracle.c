@@ -37,6 +37,15 @@
  *   R8 "round" = round half to even.
  *   R9 Epilogue: y = fp16( ((f32(acc)*s_tok[t]) * s_grp[group(o)]) + f32(bias[o]) ),
  *      each a separate IEEE round-to-nearest op (no contraction).
+ *   R12 Bias-add + quant (the token quantization fused into a bias-add,
+ *      "Kernel fusion for token-wise activation quantization"): v = f32(x) +
+ *      f32(bias), one fp32 add; y = fp16(v); then the token quantization.
+ *   R13 GeLU + quant: GeLU is its exact form, gelu(v) = v * Phi(v) =
+ *      0.5 v (1 + erf(v / sqrt 2)) = 0.5 v erfc(-v / sqrt 2), on v of R12;
+ *      y = fp16(gelu(v)).  Here it is evaluated in double (erfc form) and
+ *      rounded once to fp16; a kernel evaluating it in fp32 (with its math
+ *      library's erfc) may differ by one fp16 ulp, and its codes are then
+ *      those of the token quantization of its own y.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
  * fp16 values cross the interface as their uint16 bit patterns.
@@ -52,6 +61,13 @@
 #endif
 
 /* ---------------------------------------------------------------- fp16 */
+
+static uint16_t d2h(double d) {
+    _Float16 h = (_Float16)d; /* one IEEE round to nearest even */
+    uint16_t bits;
+    memcpy(&bits, &h, 2);
+    return bits;
+}
 
 static float h2f(uint16_t bits) {
     _Float16 h;
@@ -302,6 +318,40 @@ int zqo_ln_quant(const uint16_t *X, const uint16_t *gamma, const uint16_t *beta,
 /* acc[t,o] = sum_k xq[t,k]*wq[o,k], summed in int64 and checked to fit
  * int32 (the INT32 accumulator of the INT8 GEMM).  Returns 0, or -2 if a
  * sum does not fit int32. */
+/* GeLU, exact form (R13), in double: v * Phi(v) with Phi(v) = 0.5 erfc(-v / sqrt 2),
+ * the same function as 0.5 v (1 + erf(v / sqrt 2)) without its cancellation
+ * for negative v. */
+double zqo_gelu(double v) { return 0.5 * v * erfc(-v / sqrt(2.0)); }
+
+/* The token quantization fused into a bias-add (act = 0) or into a GeLU
+ * (act = 1), R12 / R13: per row, y = fp16(act(f32(x) + f32(bias))), then
+ * absmax -> scale -> codes exactly as zqo_token_quant.  bias and Y may be
+ * NULL. */
+int zqo_bias_act_quant(const uint16_t *X, const uint16_t *bias, int T, int K, int act, int8_t *q,
+                       float *s_tok, uint16_t *Y) {
+    if (T < 0 || K < 1 || act < 0 || act > 1) return -1;
+    uint16_t *row = (uint16_t *)malloc((size_t)K * 2);
+    if (!row) return -1;
+    for (int t = 0; t < T; ++t) {
+        const uint16_t *x = X + (size_t)t * K;
+        float amax = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float v = h2f(x[k]);
+            if (bias) v = v + h2f(bias[k]);
+            const uint16_t yb = act == 1 ? d2h(zqo_gelu((double)v)) : f2h(v);
+            row[k] = yb;
+            float a = fabsf(h2f(yb));
+            if (a > amax) amax = a;
+        }
+        float inv;
+        s_tok[t] = eq2_scale(amax, 127, &inv);
+        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(row[k]), inv, 127);
+        if (Y) memcpy(Y + (size_t)t * K, row, (size_t)K * 2);
+    }
+    free(row);
+    return 0;
+}
+
 int zqo_gemm_i32(const int8_t *xq, const int8_t *wq, int T, int N, int K, int32_t *acc) {
     for (int t = 0; t < T; ++t)
         for (int o = 0; o < N; ++o) {

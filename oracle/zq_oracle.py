@@ -69,11 +69,14 @@ def _bind(lib):
     lib.zqo_token_quant.argtypes = [P, I, I, P, P]
     lib.zqo_ln_quant.argtypes = [P, P, P, I, I, ctypes.c_float, P, P, P]
     lib.zqo_gemm_i32.argtypes = [P, P, I, I, I, P]
+    lib.zqo_gelu.argtypes = [ctypes.c_double]
+    lib.zqo_gelu.restype = ctypes.c_double
+    lib.zqo_bias_act_quant.argtypes = [P, P, I, I, I, P, P, P]
     lib.zqo_dequant.argtypes = [P, P, P, I, P, I, I, P]
     lib.zqo_linear_q.argtypes = [P, P, P, P, I, P, I, I, I, P]
     lib.zqo_rounding_is_nearest.argtypes = []
     for f in ("zqo_quantize_weights_groupwise", "zqo_pack_int4", "zqo_unpack_int4",
-              "zqo_layernorm", "zqo_token_quant", "zqo_ln_quant", "zqo_gemm_i32",
+              "zqo_layernorm", "zqo_token_quant", "zqo_ln_quant", "zqo_bias_act_quant", "zqo_gemm_i32",
               "zqo_dequant", "zqo_linear_q", "zqo_rounding_is_nearest"):
         getattr(lib, f).restype = I
     return lib
@@ -188,6 +191,29 @@ def ln_quant(X, gamma=None, beta=None, eps: float = 1e-5, want_y: bool = False):
     return (q, s, y) if want_y else (q, s)
 
 
+ACT_NONE, ACT_GELU = 0, 1
+
+
+def gelu(v: float) -> float:
+    """GeLU, exact (erf) form, in double (reading R13)."""
+    return float(_L().zqo_gelu(float(v)))
+
+
+def bias_act_quant(X, bias=None, act: int = ACT_NONE, want_y: bool = False):
+    """The token quantization fused into a bias-add (act = ACT_NONE) or a GeLU
+    (act = ACT_GELU) (Sec. 3.4 "Kernel fusion for token-wise activation
+    quantization"; readings R12 / R13).  Returns (q, s_tok) or (q, s_tok, y)."""
+    X = _h(X)
+    T, K = X.shape
+    q = np.empty((T, K), np.int8)
+    s = np.empty(T, np.float32)
+    y = np.empty((T, K), np.float16) if want_y else None
+    b = None if bias is None else _h(bias, (K,))
+    _check(_L().zqo_bias_act_quant(_p(X), _p(b), T, K, int(act), _p(q), _p(s), _p(y)),
+           "bias_act_quant")
+    return (q, s, y) if want_y else (q, s)
+
+
 def gemm_i32(xq, wq):
     """INT8 x INT8 -> INT32 accumulator, acc[t,o] = sum_k xq[t,k]*wq[o,k]
     (Sec. 3.4 "Dequantization fused into the GEMM epilogue": the INT32 result)."""
@@ -234,6 +260,6 @@ def rounding_is_nearest() -> bool:
 
 __all__ = [
     "build", "group_of", "group_index", "quantize_weights_groupwise", "pack_int4", "unpack_int4",
-    "ln_row_stats", "layernorm", "token_quant", "ln_quant", "gemm_i32", "dequant",
-    "linear_q", "rounding_is_nearest",
+    "ln_row_stats", "layernorm", "token_quant", "ln_quant", "ACT_NONE", "ACT_GELU", "gelu",
+    "bias_act_quant", "gemm_i32", "dequant", "linear_q", "rounding_is_nearest",
 ]

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(zq):
 
 
 def test_status_strings_and_version(zq):
-    assert zq.abi_version() == 100
+    assert zq.abi_version() == 101
     for s in range(7):
         assert zq.status_str(s).startswith("ZQ_")
     assert "unknown" in zq.status_str(99)
@@ -98,7 +98,25 @@ def test_ln_quant_rejects(zq, args, expect):
     assert rc == getattr(zq, "ZQ_ERR_" + expect)
 
 
+@pytest.mark.parametrize("args,expect", [
+    # (X, bias, T, K, act, Xq, s_tok, Y_act)
+    ((FAKE, None, 4, 64, 2, FAKE, FAKE, None), "UNSUPPORTED"),
+    ((FAKE, None, 4, 64, -1, FAKE, FAKE, None), "UNSUPPORTED"),
+    ((FAKE, None, 4, 40, 1, FAKE, FAKE, None), "SHAPE"),
+    ((FAKE, None, 4, 65536, 0, FAKE, FAKE, None), "SHAPE"),
+    ((FAKE, None, -1, 64, 0, FAKE, FAKE, None), "SHAPE"),
+    ((None, None, 4, 64, 1, FAKE, FAKE, None), "NULL"),
+    ((FAKE, None, 4, 64, 1, FAKE, None, None), "NULL"),
+    ((FAKE, FAKE + 8, 4, 64, 0, FAKE, FAKE, None), "ALIGN"),
+    ((FAKE, None, 4, 64, 1, FAKE, FAKE, FAKE + 2), "ALIGN"),
+])
+def test_bias_act_quant_rejects(zq, args, expect):
+    rc = zq.lib().zq_bias_act_quant(*args, None)
+    assert rc == getattr(zq, "ZQ_ERR_" + expect)
+
+
 def test_zero_tokens_is_a_no_op(zq):
+    assert zq.lib().zq_bias_act_quant(None, None, 0, 64, 1, None, None, None, None) == zq.ZQ_OK
     assert zq.lib().zq_ln_quant(None, None, None, 0, 64, 1e-5, None, None, None, None) == zq.ZQ_OK
     for fn in ("zq_gemm_w8a8", "zq_gemm_w4a8"):
         assert getattr(zq.lib(), fn)(None, None, None, None, 4, None, 0, 256, 64, None, None,

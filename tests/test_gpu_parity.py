@@ -249,6 +249,58 @@ def test_gemm_zero_scales_give_bias(zq):
     assert_bits_equal(Y, np.broadcast_to(b, (T, N)))
 
 
+# ------------------------------------------------------------ bias-add / GeLU + quant
+
+ACT_SHAPES = [(5, 16), (37, 768), (64, 3072), (9, 4096), (3, 16384), (130, 1040)]
+
+
+def _run_act(zq, X, b, act):
+    T, K = X.shape
+    y = torch.empty((T, K), dtype=torch.float16, device="cuda")
+    xq, st = zq.bias_act_quant(dev(torch.from_numpy(X)), None if b is None else dev(torch.from_numpy(b)),
+                               act, y=y)
+    return host(xq), host(st), host(y)
+
+
+@pytest.mark.parametrize("T,K", ACT_SHAPES)
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_bias_quant_bit_exact(zq, T, K, with_bias):
+    """Token quantization fused into a bias-add: every output bit equals the
+    oracle's (one fp32 add, fp16 rounding, Eq. 2)."""
+    rng = np.random.default_rng(T * 31 + K)
+    X = synth.activations(T, K, seed=T + K, n_outliers=6, outlier_scale=20.0).numpy()
+    X[0, :8] = np.array([-0.0, 0.0, 65504, -65504, 6e-8, -6e-8, 1.0, -1.0], np.float16)
+    b = None
+    if with_bias:
+        b = (rng.standard_normal(K) * 2).astype(np.float16)
+        b[2:4] = 0  # keep x + b finite next to +-65504
+    q, s, y = _run_act(zq, X, b, zq.ACT_NONE)
+    q_ref, s_ref, y_ref = oracle.bias_act_quant(X, b, oracle.ACT_NONE, want_y=True)
+    assert_bits_equal(y, y_ref)
+    assert_bits_equal(q, q_ref)
+    assert_bits_equal(s, s_ref)
+
+
+@pytest.mark.parametrize("T,K", ACT_SHAPES)
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gelu_quant_matches_oracle(zq, T, K, with_bias):
+    """Token quantization fused into a GeLU: y (CUDA's erfcf in fp32) is
+    within one fp16 ulp of the oracle's y (fp64, rounded once), and the codes
+    and scales are exactly the token quantization of the kernel's own y."""
+    rng = np.random.default_rng(T * 17 + K)
+    X = (rng.standard_normal((T, K)) * 3).astype(np.float16)
+    X[0, :6] = np.array([-0.0, 0.0, -12.0, 12.0, -3.0, 3.0], np.float16)
+    b = (rng.standard_normal(K) * 0.5).astype(np.float16) if with_bias else None
+    q, s, y = _run_act(zq, X, b, zq.ACT_GELU)
+    _, _, y_ref = oracle.bias_act_quant(X, b, oracle.ACT_GELU, want_y=True)
+    d = np.abs(y.astype(np.float64) - y_ref.astype(np.float64))
+    assert np.all(d <= ulp16(y_ref)), f"max |dy| {d.max()}"
+    assert np.mean(y.view(np.uint16) == y_ref.view(np.uint16)) > 0.99
+    q_own, s_own = oracle.token_quant(y)
+    assert_bits_equal(q, q_own)
+    assert_bits_equal(s, s_own)
+
+
 # ------------------------------------------------------------ matrix-vector path (T <= 4)
 
 @pytest.mark.parametrize("bits", [8, 4])

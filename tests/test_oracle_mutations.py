@@ -34,6 +34,11 @@ MUTATIONS = {
                               "v = v + (bias ? h2f(bias[N - 1 - o]) : 0.0f);\n            Y[(size_t)t * N + o] = f2h(v);\n        }\n    return 0;\n}\n\n/* GEMM"),
     "token_clamp_126": ("s_tok[t] = eq2_scale(amax, 127, &inv);\n        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(y[k]), inv, 127);",
                         "s_tok[t] = eq2_scale(amax, 127, &inv);\n        for (int k = 0; k < K; ++k) q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(y[k]), inv, 126);"),
+    "gelu_sqrt2_inverted": ("erfc(-v / sqrt(2.0))", "erfc(-v * sqrt(2.0))"),
+    "gelu_no_half": ("return 0.5 * v * erfc", "return v * erfc"),
+    "gelu_sign_flipped": ("erfc(-v / sqrt(2.0))", "erfc(v / sqrt(2.0))"),
+    "act_bias_ignored": ("if (bias) v = v + h2f(bias[k]);", "if (bias) v = v + 0.0f * h2f(bias[k]);"),
+    "act_gelu_skipped": ("act == 1 ? d2h(zqo_gelu((double)v)) : f2h(v)", "act == 1 ? f2h(v) : f2h(v)"),
 }
 
 

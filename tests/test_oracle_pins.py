@@ -398,3 +398,78 @@ def test_w48_footprint_is_about_three_times_smaller():
         q_bytes += packed.nbytes + sc.nbytes
         fp16_bytes += W.nbytes
     assert abs(fp16_bytes / q_bytes - d["w48_vs_fp16_ratio"]) < 0.01 * d["w48_vs_fp16_ratio"]
+
+
+# ------------------------------------------------ bias-add / GeLU + quant (R12, R13)
+
+def test_gelu_textbook_values_and_identity():
+    """GeLU(v) = v * Phi(v): against the standard normal CDF of an independent
+    library, the tabulated Phi(1), and the exact identity
+    gelu(v) - gelu(-v) = v * (Phi(v) + Phi(-v)) = v."""
+    from scipy.stats import norm
+    assert oracle.gelu(0.0) == 0.0
+    assert oracle.gelu(1.0) == pytest.approx(0.8413447460685429, rel=1e-14)
+    assert oracle.gelu(-1.0) == pytest.approx(-0.15865525393145707, rel=1e-13)
+    for v in np.linspace(-9.0, 9.0, 181):
+        assert oracle.gelu(v) == pytest.approx(v * norm.cdf(v), rel=1e-12, abs=1e-300)
+        assert oracle.gelu(v) - oracle.gelu(-v) == pytest.approx(v, rel=1e-14, abs=1e-15)
+
+
+def test_bias_act_quant_reduces_to_token_quant():
+    rng = np.random.default_rng(5)
+    X = (rng.standard_normal((6, 96)) * 3).astype(np.float16)
+    q0, s0 = oracle.token_quant(X)
+    # no bias: y is x bit for bit (also -0)
+    q, s, y = oracle.bias_act_quant(X, None, oracle.ACT_NONE, want_y=True)
+    assert np.array_equal(y.view(np.uint16), X.view(np.uint16))
+    assert np.array_equal(q, q0) and np.array_equal(s, s0)
+    # a zero bias: the same values (x + 0 only turns -0 into +0)
+    q, s, y = oracle.bias_act_quant(X, np.zeros(96, np.float16), oracle.ACT_NONE, want_y=True)
+    assert np.array_equal(y.astype(np.float32), X.astype(np.float32))
+    assert np.array_equal(q, q0) and np.array_equal(s, s0)
+    # a bias that cancels every value: y = 0, scale 0, codes 0
+    q, s, y = oracle.bias_act_quant(X[:1], -X[0], oracle.ACT_NONE, want_y=True)
+    assert not np.any(y.astype(np.float32)) and s[0] == 0.0 and not np.any(q)
+
+
+def test_bias_add_on_integers_is_exact():
+    """Small integers are exact in fp16 and fp32, so y = x + b exactly."""
+    rng = np.random.default_rng(6)
+    xi = rng.integers(-200, 200, (4, 64))
+    bi = rng.integers(-50, 50, 64)
+    q, s, y = oracle.bias_act_quant(xi.astype(np.float16), bi.astype(np.float16), oracle.ACT_NONE,
+                                    want_y=True)
+    assert np.array_equal(y.astype(np.int64), xi + bi)
+    amax = np.abs(xi + bi).max(axis=1).astype(np.float32)
+    assert np.array_equal(s, amax / np.float32(127))
+
+
+def test_gelu_quant_limits_and_bias_before_gelu():
+    # v >= 8: Phi(v) = 1 - 6e-16, so gelu(v) rounds to v in fp16 and the
+    # codes are those of x; v <= -10: gelu(v) is -v*Phi(v) ~ -8e-23, fp16 -0
+    big = np.array([[8.0, 9.5, 12.0, 100.0, 1000.0, 60000.0, 8.0, 17.0]], np.float16)
+    q, s, y = oracle.bias_act_quant(big, None, oracle.ACT_GELU, want_y=True)
+    assert np.array_equal(y, big)
+    assert np.array_equal(q, oracle.token_quant(big)[0])
+    neg = np.full((1, 16), -10.0, np.float16)
+    q, s, y = oracle.bias_act_quant(neg, None, oracle.ACT_GELU, want_y=True)
+    assert not np.any(y.astype(np.float32)) and s[0] == 0.0 and not np.any(q)
+    # the bias is added before the GeLU: x = 2, b = -2 gives gelu(0) = 0
+    x = np.full((1, 16), 2.0, np.float16)
+    q, s, y = oracle.bias_act_quant(x, np.full(16, -2.0, np.float16), oracle.ACT_GELU, want_y=True)
+    assert not np.any(y.astype(np.float32))
+
+
+def test_gelu_quant_moderate_values_against_normal_cdf():
+    """y is the fp16 value nearest v * Phi(v) (Phi from an independent library,
+    in fp64), and the codes are the token quantization of y."""
+    from scipy.stats import norm
+    rng = np.random.default_rng(7)
+    X = (rng.standard_normal((5, 128)) * 2).astype(np.float16)
+    b = (rng.standard_normal(128) * 0.5).astype(np.float16)
+    q, s, y = oracle.bias_act_quant(X, b, oracle.ACT_GELU, want_y=True)
+    v = X.astype(np.float32) + b.astype(np.float32)  # one fp32 add per element
+    ref = (v.astype(np.float64) * norm.cdf(v.astype(np.float64))).astype(np.float16)
+    assert np.array_equal(y, ref)
+    q2, s2 = oracle.token_quant(y)
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)

@@ -116,6 +116,21 @@ zq_status zq_bias_act_quant(const void* X, const void* bias, int T, int K, int a
                             float* s_tok, void* Y_act, zq_stream_t stream);
 
 /*
+ * zq_static_quant -- static (per-tensor) INT8 activation quantization, the
+ * prior post-training scheme the pages contrast with token-wise quantization
+ * (Sec. 3.4 "Token-wise Activation Quantization": a scale calibrated offline
+ * and frozen).  For comparison with zq_ln_quant's quant-only mode.
+ *   X      fp16 [T][K].
+ *   amax   the calibrated range A (0 <= A <= 65504), e.g. moving averages of
+ *          calibration batches' max and min, A = max(|x_max|, |x_min|).
+ *   Xq     int8 [T][K]: clamp(rne(x * (127/A)), -127, 127) (0 when A = 0).
+ *   s_tok  fp32 [T]: A/127 for every token, so the GEMMs consume it unchanged.
+ * Requirements: as zq_ln_quant (pointers X and Xq 16-byte aligned).
+ */
+zq_status zq_static_quant(const void* X, int T, int K, float amax, int8_t* Xq, float* s_tok,
+                          zq_stream_t stream);
+
+/*
  * zq_gemm_w8a8 -- INT8 x INT8 GEMM with the dequantization fused into the
  * epilogue (Sec. 3.4 "CUTLASS INT8 GEMM" and "Dequantization fused into the
  * GEMM epilogue"; Fig. 2 right, second box).

@@ -152,8 +152,9 @@ template <int W, int VPT>
 __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 32) : 8) / 2)
     ln_quant_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
                     const __half* __restrict__ beta, const __half* __restrict__ act_bias,
-                    int act, int T, int K, float eps, int8_t* __restrict__ Xq,
-                    float* __restrict__ s_tok, __half* __restrict__ Y_ln) {
+                    int act, float static_amax, int T, int K, float eps,
+                    int8_t* __restrict__ Xq, float* __restrict__ s_tok,
+                    __half* __restrict__ Y_ln) {
   constexpr int RT = 32 * W;                // threads per row
   constexpr int RPB = W >= 8 ? 1 : 8 / W;   // rows per block
   constexpr int NBLK = W * (VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4));
@@ -283,14 +284,19 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
 #pragma unroll
       for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h[e]));
     }
-    float amax = fmaxf(__low2float(m2), __high2float(m2));
-    amax = warp_max(amax);
-    if (W > 1) {
-      if (lane == 0) red_m[slot][warp_in_row] = amax;
-      __syncthreads();
+    // static quantization: one calibrated range for every token (codes may
+    // then exceed the range and are clamped), no per-row reduction
+    const bool is_static = static_amax >= 0.0f;  // uniform over the grid
+    float amax = static_amax;
+    if (!is_static) {
+      amax = warp_max(fmaxf(__low2float(m2), __high2float(m2)));
+      if (W > 1) {
+        if (lane == 0) red_m[slot][warp_in_row] = amax;
+        __syncthreads();
 #pragma unroll
-      for (int w = 0; w < W; ++w) amax = fmaxf(amax, red_m[slot][w]);
-      __syncthreads();  // red1 / red2 / red_m are reused by the next row
+        for (int w = 0; w < W; ++w) amax = fmaxf(amax, red_m[slot][w]);
+        __syncthreads();  // red1 / red2 / red_m are reused by the next row
+      }
     }
     const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
     if (valid) {
@@ -305,8 +311,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __half22float2(h[e]);
-            c[2 * e] = token_code(f.x, inv);
-            c[2 * e + 1] = token_code(f.y, inv);
+            c[2 * e] = is_static ? quant_code(f.x, inv, 127.0f) : token_code(f.x, inv);
+            c[2 * e + 1] = is_static ? quant_code(f.y, inv, 127.0f) : token_code(f.y, inv);
           }
           uint2 out;
           out.x = pack4(c[0], c[1], c[2], c[3]);
@@ -321,7 +327,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
 
 template <int W, int VPT>
 cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, const __half* ab, int act,
-                      int T, int K, float eps, int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
+                      float sa, int T, int K, float eps, int8_t* Xq, float* s, __half* Y,
+                      cudaStream_t st) {
   constexpr int RPB = W >= 8 ? 1 : 8 / W;
   constexpr int threads = RPB * 32 * W;
   int per_sm = 0;
@@ -332,40 +339,41 @@ cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, const _
   int need = (T + RPB - 1) / RPB;
   int grid = num_sms() * per_sm;
   if (grid > need) grid = need;
-  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, ab, act, T,
-                 K, eps, Xq, s, Y);
+  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, ab, act, sa,
+                 T, K, eps, Xq, s, Y);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int W>
 cudaError_t launch_ln_w(int vpt, const __half* X, const __half* g, const __half* b,
-                        const __half* ab, int act, int T, int K, float eps, int8_t* Xq, float* s,
-                        __half* Y, cudaStream_t st) {
+                        const __half* ab, int act, float sa, int T, int K, float eps, int8_t* Xq,
+                        float* s, __half* Y, cudaStream_t st) {
   switch (vpt) {
-    case 1: return launch_ln<W, 1>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
-    case 2: return launch_ln<W, 2>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
-    case 3: return launch_ln<W, 3>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
-    default: return launch_ln<W, 4>(X, g, b, ab, act, T, K, eps, Xq, s, Y, st);
+    case 1: return launch_ln<W, 1>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
+    case 2: return launch_ln<W, 2>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
+    case 3: return launch_ln<W, 3>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
+    default: return launch_ln<W, 4>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
   }
 }
 
 // Warps per row so that each thread keeps at most 4 vectors of 8 halves;
-// act < 0 selects the LayerNorm (gamma non-NULL) or quant-only form.
+// act < 0 selects the LayerNorm (gamma non-NULL) or quant-only form;
+// sa >= 0 is a static range (one scale for every token).
 cudaError_t launch_row_quant(const __half* xg, const __half* gg, const __half* bg,
-                             const __half* ab, int act, int T, int K, float eps, int8_t* Xq,
-                             float* s_tok, __half* yg, cudaStream_t st) {
+                             const __half* ab, int act, float sa, int T, int K, float eps,
+                             int8_t* Xq, float* s_tok, __half* yg, cudaStream_t st) {
   const int nvec = K / 8;
   int W = 1;
   while (W < 32 && 32 * W * 4 < nvec) W *= 2;
   const int vpt = (nvec + 32 * W - 1) / (32 * W);
   switch (W) {
-    case 1: return launch_ln_w<1>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
-    case 2: return launch_ln_w<2>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
-    case 4: return launch_ln_w<4>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
-    case 8: return launch_ln_w<8>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
-    case 16: return launch_ln_w<16>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
-    default: return launch_ln_w<32>(vpt, xg, gg, bg, ab, act, T, K, eps, Xq, s_tok, yg, st);
+    case 1: return launch_ln_w<1>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
+    case 2: return launch_ln_w<2>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
+    case 4: return launch_ln_w<4>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
+    case 8: return launch_ln_w<8>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
+    case 16: return launch_ln_w<16>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
+    default: return launch_ln_w<32>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
   }
 }
 
@@ -448,7 +456,8 @@ extern "C" zq_status zq_ln_quant(const void* X, const void* gamma, const void* b
   const __half* bg = gamma ? static_cast<const __half*>(beta) : nullptr;
   __half* yg = static_cast<__half*>(Y_ln);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const cudaError_t e = launch_row_quant(xg, gg, bg, nullptr, -1, T, K, eps, Xq, s_tok, yg, st);
+  const cudaError_t e =
+      launch_row_quant(xg, gg, bg, nullptr, -1, -1.0f, T, K, eps, Xq, s_tok, yg, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 
@@ -463,8 +472,21 @@ extern "C" zq_status zq_bias_act_quant(const void* X, const void* bias, int T, i
       (Y_act && !aligned16(Y_act)))
     return ZQ_ERR_ALIGN;
   const cudaError_t e = launch_row_quant(
-      static_cast<const __half*>(X), nullptr, nullptr, static_cast<const __half*>(bias), act, T,
-      K, 0.0f, Xq, s_tok, static_cast<__half*>(Y_act), reinterpret_cast<cudaStream_t>(stream));
+      static_cast<const __half*>(X), nullptr, nullptr, static_cast<const __half*>(bias), act, -1.0f,
+      T, K, 0.0f, Xq, s_tok, static_cast<__half*>(Y_act), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+extern "C" zq_status zq_static_quant(const void* X, int T, int K, float amax, int8_t* Xq,
+                                     float* s_tok, zq_stream_t stream) {
+  if (!(amax >= 0.0f) || amax > 65504.0f) return ZQ_ERR_SHAPE;  // also rejects NaN
+  if (T < 0 || K < 16 || K > 32768 || K % 16 != 0) return ZQ_ERR_SHAPE;
+  if (T == 0) return ZQ_OK;
+  if (!X || !Xq || !s_tok) return ZQ_ERR_NULL;
+  if (!aligned16(X) || !aligned16(Xq)) return ZQ_ERR_ALIGN;
+  const cudaError_t e = launch_row_quant(static_cast<const __half*>(X), nullptr, nullptr, nullptr,
+                                         -1, amax, T, K, 0.0f, Xq, s_tok, nullptr,
+                                         reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 

@@ -23,7 +23,7 @@ from int4_quantized_transformer_b200 import synth, zq
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", choices=["gemm", "ln", "act", "wquant"], default="gemm")
+    ap.add_argument("--kind", choices=["gemm", "ln", "act", "static", "wquant"], default="gemm")
     ap.add_argument("--act", choices=["gelu", "none"], default="gelu",
                     help="--kind act: GeLU + quant, or bias-add + quant (with a bias)")
     ap.add_argument("--layer", default="bert_base", choices=sorted(synth.LAYERS))
@@ -70,6 +70,8 @@ def main():
             gemm(Xq, st, Wq, sg, b, Y=Y)
         elif a.kind == "ln":
             zq.ln_quant(X, gamma, beta, Xq=Xq, s_tok=st)
+        elif a.kind == "static":
+            zq.static_quant(X, 8.0, Xq=Xq, s_tok=st)
         elif a.kind == "act":
             zq.bias_act_quant(X, act_bias, zq.ACT_GELU if a.act == "gelu" else zq.ACT_NONE,
                               Xq=Xq, s_tok=st)
@@ -106,7 +108,7 @@ def main():
     ops = 2.0 * T * s.N * s.K
     res = {"kind": a.kind, "layer": a.layer, "gemm": s.name, "T": T, "N": s.N, "K": s.K,
            "bits": s.bits, "us": round(us, 2)}
-    if a.kind in ("ln", "act"):  # fp16 in, int8 + one fp32 scale per row out
+    if a.kind in ("ln", "act", "static"):  # fp16 in, int8 + one fp32 scale per row out
         res["gbs"] = round((3 * T * s.K + 4 * T) / us / 1e3, 1)
     else:
         res["tops"] = round(ops / us / 1e6, 1)

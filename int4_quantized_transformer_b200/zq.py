@@ -23,7 +23,7 @@ OPT_GEMM_PATH, OPT_GEMM_BN, OPT_SPLIT_K, OPT_MAX_CTAS, OPT_CTA_PAIR = 1, 2, 3, 4
 EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
-    "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant",
+    "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant", "zq_static_quant",
 )
 
 
@@ -52,6 +52,7 @@ def _load():
         "zq_debug_wait_timeout": ([P], I),
         "zq_gemm_w8a8_noalloc": ([P, P, P, P, I, P, I, I, I, P, P, P], I),
         "zq_bias_act_quant": ([P, P, I, I, I, P, P, P, P], I),
+        "zq_static_quant": ([P, I, I, F, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -184,6 +185,20 @@ def bias_act_quant(X: torch.Tensor, bias=None, act: int = ACT_NONE, Xq=None, s_t
         _dev(X, torch.float16, (T, K), "X"), _dev(bias, torch.float16, (K,), "bias"), T, K,
         int(act), _dev(Xq, torch.int8, (T, K), "Xq"), _dev(s_tok, torch.float32, (T,), "s_tok"),
         _dev(y, torch.float16, (T, K), "Y_act"), _stream(stream)), "zq_bias_act_quant")
+    return Xq, s_tok
+
+
+def static_quant(X: torch.Tensor, amax: float, Xq=None, s_tok=None, stream=None):
+    """Static (per-tensor) INT8 quantization with a calibrated range amax
+    (zq_static_quant).  Returns (Xq int8 [T,K], s_tok fp32 [T] = amax/127)."""
+    T, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
+    if s_tok is None:
+        s_tok = torch.empty(T, dtype=torch.float32, device=X.device)
+    _check(_lib.zq_static_quant(
+        _dev(X, torch.float16, (T, K), "X"), T, K, float(amax), _dev(Xq, torch.int8, (T, K), "Xq"),
+        _dev(s_tok, torch.float32, (T,), "s_tok"), _stream(stream)), "zq_static_quant")
     return Xq, s_tok
 
 

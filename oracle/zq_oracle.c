@@ -46,6 +46,12 @@
  *      rounded once to fp16; a kernel evaluating it in fp32 (with its math
  *      library's erfc) may differ by one fp16 ulp, and its codes are then
  *      those of the token quantization of its own y.
+ *   R14 Static (per-tensor) activation quantization, the prior PTQ scheme the
+ *      pages contrast with token-wise quantization: calibration keeps
+ *      moving averages x_max = m x_max + (1-m) max(batch), x_min likewise
+ *      (m = 0.95), started from the first batch's max and min, fp32; the
+ *      range is A = max(|x_max|, |x_min|); every token then uses
+ *      s = A/127 and q = clamp(rne(x * (127/A)), -127, 127).
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
  * fp16 values cross the interface as their uint16 bit patterns.
@@ -349,6 +355,45 @@ int zqo_bias_act_quant(const uint16_t *X, const uint16_t *bias, int T, int K, in
         if (Y) memcpy(Y + (size_t)t * K, row, (size_t)K * 2);
     }
     free(row);
+    return 0;
+}
+
+/* Static calibration (R14) over nb batches of T x K stored one after the
+ * other; writes the calibrated range A. */
+int zqo_static_calibrate(const uint16_t *X, int nb, int T, int K, float momentum, float *A) {
+    if (nb < 1 || T < 1 || K < 1) return -1;
+    float xmax = 0.0f, xmin = 0.0f;
+    for (int b = 0; b < nb; ++b) {
+        const uint16_t *x = X + (size_t)b * T * K;
+        float bmax = h2f(x[0]), bmin = h2f(x[0]);
+        for (size_t i = 1; i < (size_t)T * K; ++i) {
+            const float v = h2f(x[i]);
+            if (v > bmax) bmax = v;
+            if (v < bmin) bmin = v;
+        }
+        if (b == 0) {
+            xmax = bmax;
+            xmin = bmin;
+        } else {
+            xmax = momentum * xmax + (1.0f - momentum) * bmax;
+            xmin = momentum * xmin + (1.0f - momentum) * bmin;
+        }
+    }
+    *A = fmaxf(fabsf(xmax), fabsf(xmin));
+    return 0;
+}
+
+/* Static quantization with the calibrated range A (R14): one scale for every
+ * token, written to s_tok so that the GEMM's dequantization is unchanged. */
+int zqo_static_quant(const uint16_t *X, int T, int K, float A, int8_t *q, float *s_tok) {
+    if (T < 0 || K < 1 || !(A >= 0.0f)) return -1;
+    float inv;
+    const float s = eq2_scale(A, 127, &inv);
+    for (int t = 0; t < T; ++t) {
+        s_tok[t] = s;
+        for (int k = 0; k < K; ++k)
+            q[(size_t)t * K + k] = (int8_t)eq2_quantize(h2f(X[(size_t)t * K + k]), inv, 127);
+    }
     return 0;
 }
 

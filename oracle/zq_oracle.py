@@ -72,11 +72,14 @@ def _bind(lib):
     lib.zqo_gelu.argtypes = [ctypes.c_double]
     lib.zqo_gelu.restype = ctypes.c_double
     lib.zqo_bias_act_quant.argtypes = [P, P, I, I, I, P, P, P]
+    lib.zqo_static_calibrate.argtypes = [P, I, I, I, ctypes.c_float, P]
+    lib.zqo_static_quant.argtypes = [P, I, I, ctypes.c_float, P, P]
     lib.zqo_dequant.argtypes = [P, P, P, I, P, I, I, P]
     lib.zqo_linear_q.argtypes = [P, P, P, P, I, P, I, I, I, P]
     lib.zqo_rounding_is_nearest.argtypes = []
     for f in ("zqo_quantize_weights_groupwise", "zqo_pack_int4", "zqo_unpack_int4",
-              "zqo_layernorm", "zqo_token_quant", "zqo_ln_quant", "zqo_bias_act_quant", "zqo_gemm_i32",
+              "zqo_layernorm", "zqo_token_quant", "zqo_ln_quant", "zqo_bias_act_quant",
+              "zqo_static_calibrate", "zqo_static_quant", "zqo_gemm_i32",
               "zqo_dequant", "zqo_linear_q", "zqo_rounding_is_nearest"):
         getattr(lib, f).restype = I
     return lib
@@ -214,6 +217,29 @@ def bias_act_quant(X, bias=None, act: int = ACT_NONE, want_y: bool = False):
     return (q, s, y) if want_y else (q, s)
 
 
+def static_calibrate(batches, momentum: float = 0.95) -> float:
+    """Static PTQ calibration (reading R14): moving averages of each batch's
+    max and min; returns the range A = max(|x_max|, |x_min|).  batches is
+    [nb, T, K] fp16."""
+    Xb = np.ascontiguousarray(batches, dtype=np.float16)
+    nb, T, K = Xb.shape
+    A = np.empty(1, np.float32)
+    _check(_L().zqo_static_calibrate(_p(Xb), nb, T, K, ctypes.c_float(momentum), _p(A)),
+           "static_calibrate")
+    return float(A[0])
+
+
+def static_quant(X, A: float):
+    """Static (per-tensor) quantization with range A (R14): every token uses
+    s = A/127.  Returns (q int8 [T,K], s_tok fp32 [T])."""
+    X = _h(X)
+    T, K = X.shape
+    q = np.empty((T, K), np.int8)
+    s = np.empty(T, np.float32)
+    _check(_L().zqo_static_quant(_p(X), T, K, ctypes.c_float(A), _p(q), _p(s)), "static_quant")
+    return q, s
+
+
 def gemm_i32(xq, wq):
     """INT8 x INT8 -> INT32 accumulator, acc[t,o] = sum_k xq[t,k]*wq[o,k]
     (Sec. 3.4 "Dequantization fused into the GEMM epilogue": the INT32 result)."""
@@ -261,5 +287,6 @@ def rounding_is_nearest() -> bool:
 __all__ = [
     "build", "group_of", "group_index", "quantize_weights_groupwise", "pack_int4", "unpack_int4",
     "ln_row_stats", "layernorm", "token_quant", "ln_quant", "ACT_NONE", "ACT_GELU", "gelu",
-    "bias_act_quant", "gemm_i32", "dequant", "linear_q", "rounding_is_nearest",
+    "bias_act_quant", "static_calibrate", "static_quant", "gemm_i32", "dequant", "linear_q",
+    "rounding_is_nearest",
 ]

@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(zq):
 
 
 def test_status_strings_and_version(zq):
-    assert zq.abi_version() == 101
+    assert zq.abi_version() == 102
     for s in range(7):
         assert zq.status_str(s).startswith("ZQ_")
     assert "unknown" in zq.status_str(99)
@@ -112,6 +112,21 @@ def test_ln_quant_rejects(zq, args, expect):
 ])
 def test_bias_act_quant_rejects(zq, args, expect):
     rc = zq.lib().zq_bias_act_quant(*args, None)
+    assert rc == getattr(zq, "ZQ_ERR_" + expect)
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (X, T, K, amax, Xq, s_tok)
+    ((FAKE, 4, 64, -1.0, FAKE, FAKE), "SHAPE"),
+    ((FAKE, 4, 64, float("nan"), FAKE, FAKE), "SHAPE"),
+    ((FAKE, 4, 64, 1e6, FAKE, FAKE), "SHAPE"),
+    ((FAKE, 4, 40, 1.0, FAKE, FAKE), "SHAPE"),
+    ((None, 4, 64, 1.0, FAKE, FAKE), "NULL"),
+    ((FAKE, 4, 64, 1.0, FAKE, None), "NULL"),
+    ((FAKE + 2, 4, 64, 1.0, FAKE, FAKE), "ALIGN"),
+])
+def test_static_quant_rejects(zq, args, expect):
+    rc = zq.lib().zq_static_quant(*args, None)
     assert rc == getattr(zq, "ZQ_ERR_" + expect)
 
 

@@ -301,6 +301,18 @@ def test_gelu_quant_matches_oracle(zq, T, K, with_bias):
     assert_bits_equal(s, s_own)
 
 
+@pytest.mark.parametrize("T,K", [(5, 16), (64, 768), (33, 3072), (7, 16384)])
+@pytest.mark.parametrize("amax", [0.0, 0.75, 3.0, 40.0])
+def test_static_quant_bit_exact(zq, T, K, amax):
+    """Static per-tensor quantization: one calibrated range for every token,
+    codes beyond it clamped; bit-exact against the oracle."""
+    X = synth.activations(T, K, seed=T + K, n_outliers=4, outlier_scale=20.0)
+    xq, st = zq.static_quant(dev(X), amax)
+    q_ref, s_ref = oracle.static_quant(X.numpy(), amax)
+    assert_bits_equal(host(xq), q_ref)
+    assert_bits_equal(host(st), s_ref)
+
+
 # ------------------------------------------------------------ matrix-vector path (T <= 4)
 
 @pytest.mark.parametrize("bits", [8, 4])

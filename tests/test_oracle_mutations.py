@@ -38,6 +38,9 @@ MUTATIONS = {
     "gelu_no_half": ("return 0.5 * v * erfc", "return v * erfc"),
     "gelu_sign_flipped": ("erfc(-v / sqrt(2.0))", "erfc(v / sqrt(2.0))"),
     "act_bias_ignored": ("if (bias) v = v + h2f(bias[k]);", "if (bias) v = v + 0.0f * h2f(bias[k]);"),
+    "static_ema_swapped": ("xmax = momentum * xmax + (1.0f - momentum) * bmax;",
+                           "xmax = (1.0f - momentum) * xmax + momentum * bmax;"),
+    "static_range_max_only": ("*A = fmaxf(fabsf(xmax), fabsf(xmin));", "*A = fabsf(xmax);"),
     "act_gelu_skipped": ("act == 1 ? d2h(zqo_gelu((double)v)) : f2h(v)", "act == 1 ? f2h(v) : f2h(v)"),
 }
 

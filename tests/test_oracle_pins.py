@@ -473,3 +473,68 @@ def test_gelu_quant_moderate_values_against_normal_cdf():
     assert np.array_equal(y, ref)
     q2, s2 = oracle.token_quant(y)
     assert np.array_equal(q, q2) and np.array_equal(s, s2)
+
+
+# ------------------------------------------------ static per-tensor quantization (R14)
+
+def test_static_calibration_moving_average():
+    """One batch: the range is max(|max|, |min|).  More batches: the moving
+    averages of the pages' Appendix B.1 formula, on values exact in fp16 and
+    fp32 (0.95 * 4 + 0.05 * 2 = 3.9 and 0.95 * (-1) + 0.05 * (-8) = -1.35)."""
+    b1 = np.array([[[1.0, -1.0, 4.0, 0.5]]], np.float16)
+    assert oracle.static_calibrate(b1) == 4.0
+    b2 = np.array([[[-3.0, 2.0, 0.0, 1.0]]], np.float16)
+    assert oracle.static_calibrate(np.concatenate([b2, b2])) == 3.0
+    x1 = np.array([[[4.0, -1.0, 0.0, 1.0]]], np.float16)
+    x2 = np.array([[[2.0, -8.0, 0.0, 1.0]]], np.float16)
+    a = oracle.static_calibrate(np.concatenate([x1, x2]), momentum=0.95)
+    assert a == pytest.approx(3.9, abs=1e-6)  # max(|3.9|, |-1.35|)
+    assert oracle.static_calibrate(np.concatenate([x2, x1]), momentum=0.95) == pytest.approx(
+        max(0.95 * 2 + 0.05 * 4, 0.95 * 8 + 0.05 * 1), abs=1e-6)
+
+
+def test_static_calibration_geometric_decay():
+    """After a first batch with range 8 and then n batches with range 2, the
+    moving average is 2 + 6 * 0.95**n (closed form of the recurrence); 100
+    iterations, the pages' calibration length, stay within fp32 rounding."""
+    first = np.full((1, 2, 8), 8.0, np.float16)
+    rest = np.full((100, 2, 8), 2.0, np.float16)
+    for n in (1, 5, 100):
+        a = oracle.static_calibrate(np.concatenate([first, rest[:n]]), momentum=0.95)
+        assert a == pytest.approx(2.0 + 6.0 * 0.95 ** n, rel=n * 1e-7)
+
+
+def test_static_quant_special_cases():
+    rng = np.random.default_rng(9)
+    X = (rng.standard_normal((1, 64)) * 3).astype(np.float16)
+    # a token whose own absmax is the calibrated range: token-wise and static agree
+    A = float(np.abs(X.astype(np.float32)).max())
+    assert all(np.array_equal(u, v) for u, v in zip(oracle.static_quant(X, A), oracle.token_quant(X)))
+    # values beyond the range saturate at +-127; a zero range gives zero codes
+    q, s = oracle.static_quant(np.array([[10.0, -10.0, 0.5, -0.5]], np.float16), 1.0)
+    assert q.tolist() == [[127, -127, 64, -64]] and s[0] == np.float32(1.0) / np.float32(127)
+    q, s = oracle.static_quant(X, 0.0)
+    assert not np.any(q) and s[0] == 0.0
+
+
+def test_token_wise_beats_static_on_varying_token_ranges():
+    """The pages' motivation for token-wise scales: with token ranges that vary
+    (here 0.25x .. 4x, the kind of variation the diagnostic reports), one
+    calibrated scale starves the small tokens.  Per-token relative L2 error of
+    the dequantized activations, on seeded synthetic data."""
+    rng = np.random.default_rng(11)
+    T, K = 256, 768
+    scale = np.exp(rng.uniform(np.log(0.25), np.log(4.0), (8, T, 1)))
+    batches = (rng.standard_normal((8, T, K)) * scale).astype(np.float16)
+    A = oracle.static_calibrate(batches[:7])      # calibrate on 7 batches
+    X = batches[7]                                # evaluate on a held-out one
+    x = X.astype(np.float64)
+    qs, ss = oracle.static_quant(X, A)
+    qt, st = oracle.token_quant(X)
+    es = np.linalg.norm(qs * ss[:, None].astype(np.float64) - x, axis=1) / np.linalg.norm(x, axis=1)
+    et = np.linalg.norm(qt * st[:, None].astype(np.float64) - x, axis=1) / np.linalg.norm(x, axis=1)
+    assert np.all(et <= es * 1.05)               # token-wise is never worse (ties up to noise)
+    small = scale[7, :, 0] < 0.5
+    assert np.median(es[small]) > 4 * np.median(et[small])
+    print(f"median per-token relative error: token-wise {np.median(et):.4f}, static {np.median(es):.4f}; "
+          f"small-range tokens: token-wise {np.median(et[small]):.4f}, static {np.median(es[small]):.4f}")

@@ -167,6 +167,41 @@ zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
                        int32_t* acc_dbg, zq_stream_t stream);
 
 /*
+ * zq_gemm_w8a16 -- the quantized linear layer with FP16 activations and
+ * group-wise INT8 weights (W8A16: the summary page's "Main Quantitative
+ * Results", Table 4; also the GPT-NeoX self-attention input that stays in
+ * FP16 while its weights are INT8, "INT4/INT8 Mixed-Precision Quantization").
+ *   X           fp16 [T][K], row-major (no activation quantization).
+ *   Wq, s_grp   int8 [N][K] and fp32 [g] from zq_quantize_weights_groupwise.
+ *   bias        fp16 [N] or NULL (= 0).
+ *   Y           fp16 [T][N]:
+ *               acc[t][o] = sum_k x[t][k] * Wq[o][k]   (fp32 accumulation on
+ *                           tcgen05 tensor cores, codes exact in fp16; the
+ *                           summation order is the hardware's)
+ *               Y[t][o] = fp16(f32(acc * s_grp[group(o)]) + f32(bias[o]))
+ *               i.e. X * (Wq * S)^T + bias with each row's group scale
+ *               applied after the K sum, where it factors out exactly.
+ *   acc_dbg     fp32 [T][N] or NULL: also store acc (for checking).
+ * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
+ * 16 <= K <= 2^20, K % 16 == 0, 1 <= g <= N, pointers 16-byte aligned.
+ * Errors: as zq_gemm_w8a8 (argument errors before any launch).
+ */
+zq_status zq_gemm_w8a16(const void* X, const int8_t* Wq, const float* s_grp, int g,
+                        const void* bias, int T, int N, int K, void* Y, float* acc_dbg,
+                        zq_stream_t stream);
+
+/*
+ * zq_gemm_w4a16 -- as zq_gemm_w8a16 with INT4 weights (the W4/8A16
+ * configurations of "INT4/INT8 Mixed-Precision Quantization": INT4 FFN
+ * weights with FP16 activations).  Wq4 is uint8 [N][K/2] in the layout of
+ * zq_quantize_weights_groupwise(bits=4); the kernel widens the nibbles to
+ * fp16 in shared memory.  Requirements as zq_gemm_w8a16, plus K % 32 == 0.
+ */
+zq_status zq_gemm_w4a16(const void* X, const uint8_t* Wq4, const float* s_grp, int g,
+                        const void* bias, int T, int N, int K, void* Y, float* acc_dbg,
+                        zq_stream_t stream);
+
+/*
  * zq_gemm_w8a8_noalloc -- zq_gemm_w8a8 for callers that must not let a
  * library allocate device memory: a serving runtime that owns the whole
  * device memory pool, a process whose memory budget is fixed up front, or
@@ -209,7 +244,9 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  *                      3 = CUDA-core matrix-vector product (T <= 4, else
  *                          ZQ_ERR_UNSUPPORTED); automatic at T <= 4 with
  *                          INT4 weights and at T <= 2 with INT8 ones.
- *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256).
+ *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256);
+ *                      the FP16-activation GEMMs accept 128 or 256 (other
+ *                      values: ZQ_ERR_UNSUPPORTED) and ignore the path.
  *   ZQ_OPT_SPLIT_K     number of K splits for path 2 (1 = none).
  *   ZQ_OPT_MAX_CTAS    cap on the number of CTAs of the GEMM (persistent grid).
  *   ZQ_OPT_CTA_PAIR    path 1: 1 = one CTA per 128 x BN

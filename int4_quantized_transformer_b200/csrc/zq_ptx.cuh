@@ -1,5 +1,6 @@
 // zq_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers with bounded
-// waits, TMA tensor loads, tcgen05 (TMEM alloc, MMA kind::i8, commit, loads).
+// waits, TMA tensor loads, tcgen05 (TMEM alloc, MMA kind::i8 and kind::f16,
+// commit, loads).
 #pragma once
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -246,6 +247,17 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, fp16 x fp16 -> fp32.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // CTA-pair MMA (issued by the even CTA of the pair): M = 256 rows, of which
 // each CTA holds 128 rows of A and N/2 rows of B at the same shared-memory
 // offsets; each CTA's TMEM receives its 128 rows of D.
@@ -315,6 +327,13 @@ __device__ __forceinline__ uint64_t make_sw128_desc(uint32_t smem_addr) {
 __host__ __device__ constexpr uint32_t make_idesc_i8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B (formats 0 at [7,10)
+// and [10,13)) and an fp32 D ([4,6) = 1), both K-major, N>>3 at [17,23),
+// M>>4 at [24,29).
+__host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 }  // namespace zq

@@ -24,6 +24,7 @@ EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
     "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant", "zq_static_quant",
+    "zq_gemm_w8a16", "zq_gemm_w4a16",
 )
 
 
@@ -53,6 +54,8 @@ def _load():
         "zq_gemm_w8a8_noalloc": ([P, P, P, P, I, P, I, I, I, P, P, P], I),
         "zq_bias_act_quant": ([P, P, I, I, I, P, P, P, P], I),
         "zq_static_quant": ([P, I, I, F, P, P, P], I),
+        "zq_gemm_w8a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
+        "zq_gemm_w4a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -234,6 +237,34 @@ def gemm_w8a8_noalloc(Xq, s_tok, Wq, s_grp, bias=None, Y=None, acc_dbg=None, str
     scratch comes from a fixed array in device memory (zq_gemm_w8a8_noalloc)."""
     return _gemm(_lib.zq_gemm_w8a8_noalloc, "zq_gemm_w8a8_noalloc", Xq, s_tok, Wq, s_grp, bias,
                  Wq.shape[0], Y, acc_dbg, stream, 8)
+
+
+def _gemm_a16(fn, what, X, Wq, s_grp, bias, N, Y, acc, stream, bits):
+    T, K = X.shape
+    g = s_grp.shape[0]
+    if Y is None:
+        Y = torch.empty((T, N), dtype=torch.float16, device=X.device)
+    wshape = (N, K) if bits == 8 else (N, K // 2)
+    _check(fn(
+        _dev(X, torch.float16, (T, K), "X"),
+        _dev(Wq, torch.int8 if bits == 8 else torch.uint8, wshape, "Wq"),
+        _dev(s_grp, torch.float32, (g,), "s_grp"), g, _dev(bias, torch.float16, (N,), "bias"),
+        T, N, K, _dev(Y, torch.float16, (T, N), "Y"), _dev(acc, torch.float32, (T, N), "acc_dbg"),
+        _stream(stream)), what)
+    return Y
+
+
+def gemm_w8a16(X, Wq, s_grp, bias=None, Y=None, acc_dbg=None, stream=None):
+    """FP16 activations, INT8 weights: Y = fp16(acc * s_grp[group] + bias),
+    acc = X Wq^T accumulated in fp32 on the tensor cores."""
+    return _gemm_a16(_lib.zq_gemm_w8a16, "zq_gemm_w8a16", X, Wq, s_grp, bias, Wq.shape[0], Y,
+                     acc_dbg, stream, 8)
+
+
+def gemm_w4a16(X, Wq4, s_grp, bias=None, Y=None, acc_dbg=None, stream=None):
+    """As gemm_w8a16 with packed INT4 weights uint8 [N, K/2]."""
+    return _gemm_a16(_lib.zq_gemm_w4a16, "zq_gemm_w4a16", X, Wq4, s_grp, bias, Wq4.shape[0], Y,
+                     acc_dbg, stream, 4)
 
 
 def debug_wait_timeout(stream=None):

@@ -52,6 +52,14 @@
  *      (m = 0.95), started from the first batch's max and min, fp32; the
  *      range is A = max(|x_max|, |x_min|); every token then uses
  *      s = A/127 and q = clamp(rne(x * (127/A)), -127, 127).
+ *   R15 FP16 activations with quantized weights (W8A16, W4/8A16; the summary
+ *      page's "Main Quantitative Results" and "INT4/INT8 Mixed-Precision
+ *      Quantization"): the layer is X (q S)^T + b with the dequantized
+ *      weights q * S[group(o)].  Evaluated here in double: acc = sum_k
+ *      x[t,k] q[o,k] (every product exact), y = acc * S + b, rounded once to
+ *      fp16.  A tensor-core kernel sums the products in fp32 in its own
+ *      order and applies S after the sum, so it agrees within a rounding
+ *      bound, not bit for bit.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -shared -fPIC.
  * fp16 values cross the interface as their uint16 bit patterns.
@@ -446,4 +454,23 @@ int zqo_linear_q(const int8_t *xq, const float *s_tok, const int8_t *wq, const f
 }
 
 /* Reports the rounding mode so a test can confirm round-to-nearest. */
+/* FP16 activations times group-wise quantized weights (R15): acc and y in
+ * double, Y = fp16(y).  q is int8 [N][K] (INT4 weights: unpacked first). */
+int zqo_gemm_a16(const uint16_t *X, const int8_t *q, const float *s_grp, int g,
+                 const uint16_t *bias, int T, int N, int K, double *acc, double *y, uint16_t *Y) {
+    if (T < 0 || N < 1 || K < 1 || g < 1 || g > N) return -1;
+    for (int t = 0; t < T; ++t)
+        for (int o = 0; o < N; ++o) {
+            double sum = 0.0;
+            for (int k = 0; k < K; ++k)
+                sum += (double)h2f(X[(size_t)t * K + k]) * (double)q[(size_t)o * K + k];
+            const double v = sum * (double)s_grp[zqo_group_of(o, N, g)] +
+                             (bias ? (double)h2f(bias[o]) : 0.0);
+            acc[(size_t)t * N + o] = sum;
+            y[(size_t)t * N + o] = v;
+            Y[(size_t)t * N + o] = d2h(v);
+        }
+    return 0;
+}
+
 int zqo_rounding_is_nearest(void) { return fegetround() == FE_TONEAREST; }

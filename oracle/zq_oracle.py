@@ -76,6 +76,7 @@ def _bind(lib):
     lib.zqo_static_quant.argtypes = [P, I, I, ctypes.c_float, P, P]
     lib.zqo_dequant.argtypes = [P, P, P, I, P, I, I, P]
     lib.zqo_linear_q.argtypes = [P, P, P, P, I, P, I, I, I, P]
+    lib.zqo_gemm_a16.argtypes = [P, P, P, I, P, I, I, I, P, P, P]
     lib.zqo_rounding_is_nearest.argtypes = []
     for f in ("zqo_quantize_weights_groupwise", "zqo_pack_int4", "zqo_unpack_int4",
               "zqo_layernorm", "zqo_token_quant", "zqo_ln_quant", "zqo_bias_act_quant",
@@ -280,6 +281,25 @@ def linear_q(xq, s_tok, wq, s_grp, bias=None):
     return Y
 
 
+def gemm_a16(X, q, s_grp, bias=None):
+    """FP16 activations times group-wise quantized weights (R15; W8A16 and,
+    with q = unpack_int4(packed), W4A16): X (q S)^T + b in double.  Returns
+    (acc float64 [T,N], y float64 [T,N], Y fp16 [T,N] = fp16(y))."""
+    X = _h(X)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    T, K = X.shape
+    N, K2 = q.shape
+    assert K == K2
+    s_grp = np.ascontiguousarray(s_grp, dtype=np.float32)
+    b = None if bias is None else _h(bias, (N,))
+    acc = np.empty((T, N), np.float64)
+    y = np.empty((T, N), np.float64)
+    Y = np.empty((T, N), np.float16)
+    _check(_L().zqo_gemm_a16(_p(X), _p(q), _p(s_grp), s_grp.size, _p(b), T, N, K, _p(acc), _p(y),
+                             _p(Y)), "gemm_a16")
+    return acc, y, Y
+
+
 def rounding_is_nearest() -> bool:
     return bool(_L().zqo_rounding_is_nearest())
 
@@ -288,5 +308,5 @@ __all__ = [
     "build", "group_of", "group_index", "quantize_weights_groupwise", "pack_int4", "unpack_int4",
     "ln_row_stats", "layernorm", "token_quant", "ln_quant", "ACT_NONE", "ACT_GELU", "gelu",
     "bias_act_quant", "static_calibrate", "static_quant", "gemm_i32", "dequant", "linear_q",
-    "rounding_is_nearest",
+    "gemm_a16", "rounding_is_nearest",
 ]

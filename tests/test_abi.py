@@ -160,6 +160,42 @@ def test_gemm_rejects(zq, fn, args, expect):
     assert rc == getattr(zq, "ZQ_ERR_" + expect)
 
 
+@pytest.mark.parametrize("fn", ["zq_gemm_w8a16", "zq_gemm_w4a16"])
+@pytest.mark.parametrize("args,expect", [
+    # (X, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg)
+    ((FAKE, FAKE, FAKE, 4, None, 16, 250, 64, FAKE, None), "SHAPE"),      # N % 8
+    ((FAKE, FAKE, FAKE, 4, None, 16, 0, 64, FAKE, None), "SHAPE"),
+    ((FAKE, FAKE, FAKE, 4, None, 16, 256, 72, FAKE, None), "SHAPE"),      # K % 16
+    ((FAKE, FAKE, FAKE, 4, None, 16, 256, (1 << 20) + 64, FAKE, None), "SHAPE"),
+    ((FAKE, FAKE, FAKE, 0, None, 16, 256, 64, FAKE, None), "SHAPE"),
+    ((FAKE, FAKE, FAKE, 257, None, 16, 256, 64, FAKE, None), "SHAPE"),
+    ((FAKE, FAKE, FAKE, 4, None, -1, 256, 64, FAKE, None), "SHAPE"),
+    ((None, FAKE, FAKE, 4, None, 16, 256, 64, FAKE, None), "NULL"),
+    ((FAKE, None, FAKE, 4, None, 16, 256, 64, FAKE, None), "NULL"),
+    ((FAKE, FAKE, None, 4, None, 16, 256, 64, FAKE, None), "NULL"),
+    ((FAKE, FAKE, FAKE, 4, None, 16, 256, 64, None, None), "NULL"),
+    ((FAKE + 2, FAKE, FAKE, 4, None, 16, 256, 64, FAKE, None), "ALIGN"),
+    ((FAKE, FAKE + 8, FAKE, 4, None, 16, 256, 64, FAKE, None), "ALIGN"),
+    ((FAKE, FAKE, FAKE, 4, FAKE + 2, 16, 256, 64, FAKE, None), "ALIGN"),
+    ((FAKE, FAKE, FAKE, 4, None, 16, 256, 64, FAKE, FAKE + 4), "ALIGN"),
+])
+def test_gemm_a16_rejects(zq, fn, args, expect):
+    rc = getattr(zq.lib(), fn)(*args, None)
+    assert rc == getattr(zq, "ZQ_ERR_" + expect)
+
+
+def test_gemm_a16_argument_rules(zq):
+    L = zq.lib()
+    # INT4 weights need K % 32 == 0
+    assert L.zq_gemm_w4a16(FAKE, FAKE, FAKE, 4, None, 16, 256, 48, FAKE, None, None) == zq.ZQ_ERR_SHAPE
+    # no tokens: nothing to check, nothing launched
+    assert L.zq_gemm_w8a16(None, None, None, 4, None, 0, 256, 64, None, None, None) == zq.ZQ_OK
+    # only the 128- and 256-wide tiles exist for FP16 activations
+    with zq.options(bn=192):
+        assert L.zq_gemm_w8a16(FAKE, FAKE, FAKE, 4, None, 16, 256, 64, FAKE, None,
+                               None) == zq.ZQ_ERR_UNSUPPORTED
+
+
 def test_w4a8_needs_k_multiple_of_32(zq):
     rc = zq.lib().zq_gemm_w4a8(FAKE, FAKE, FAKE, FAKE, 4, None, 16, 256, 48, FAKE, None, None)
     assert rc == zq.ZQ_ERR_SHAPE

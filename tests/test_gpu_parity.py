@@ -402,6 +402,123 @@ def test_full_size_sampled_rows(zq, layer, gi, T):
     assert_fp16_close(host(Y_d)[rows], oracle.dequant(acc, st, sg, inp.b.numpy()))
 
 
+# ------------------------------------------------------------ FP16 activations (W8A16 / W4A16)
+#
+# The tensor cores sum fp16 x code products in fp32 in their own order, so the
+# GPU accumulator is compared with the oracle's double sum within the bound of
+# fp32 summation in any order, |acc - acc64| <= 2 K 2^-24 sum_k |x q| (the
+# factor 2 also covers adders that truncate), and Y within that bound times
+# the group scale, plus the two fp32 roundings of the epilogue and half an
+# fp16 ulp for the final rounding.
+
+def _assert_a16_close(X, q, sg, acc, Y, acc_ref, y_ref, Y_ref, min_equal=0.8):
+    T, K = X.shape
+    N = q.shape[0]
+    mag = np.abs(X.astype(np.float64)) @ np.abs(q.astype(np.float64)).T
+    e_acc = 2.0 * K * 2.0 ** -24 * mag
+    bad = np.abs(acc.astype(np.float64) - acc_ref) > e_acc
+    assert not bad.any(), f"{bad.sum()} accumulators outside the fp32 summation bound"
+    s = sg.astype(np.float64)[np.arange(N) * sg.size // N][None, :]
+    y = Y.astype(np.float64)
+    tol = (e_acc * s + 2.0 ** -23 * (np.abs(acc_ref * s) + np.abs(y_ref))
+           + 0.5 * ulp16(np.maximum(np.abs(y), np.abs(y_ref))))
+    bad = np.abs(y - y_ref) > tol
+    assert not bad.any(), f"{bad.sum()} fp16 outputs outside the tolerance"
+    equal = np.mean(Y.view(np.uint16) == Y_ref.view(np.uint16))
+    assert equal >= min_equal, f"only {equal:.3f} of the outputs equal the correctly rounded value"
+
+
+def _check_a16(zq, T, N, K, g, bits, seed=0, bias=True, **opts):
+    X = synth.activations(T, K, seed=seed, n_outliers=6, outlier_scale=20.0)
+    W = synth.weights(N, K, 0.02, seed=seed + 1)
+    b = synth.bias(N, seed + 2) if bias else None
+    wq, sg = oracle.quantize_weights_groupwise(W.numpy(), g, bits)
+    wdev = torch.from_numpy(oracle.pack_int4(wq) if bits == 4 else wq).cuda()
+    acc_d = torch.empty((T, N), dtype=torch.float32, device="cuda")
+    fn = zq.gemm_w4a16 if bits == 4 else zq.gemm_w8a16
+    with zq.options(**opts):
+        Y = fn(dev(X), wdev, torch.from_numpy(sg).cuda(), None if b is None else dev(b),
+               acc_dbg=acc_d)
+    acc_ref, y_ref, Y_ref = oracle.gemm_a16(X.numpy(), wq, sg, None if b is None else b.numpy())
+    _assert_a16_close(X.numpy(), wq, sg, host(acc_d), host(Y), acc_ref, y_ref, Y_ref)
+
+
+A16_SHAPES = [
+    # T, N, K, g
+    (16, 256, 64, 4),
+    (1, 256, 64, 4),
+    (7, 768, 768, 48),
+    (129, 1024, 768, 48),  # ragged token tile
+    (300, 768, 784, 48),   # K not a multiple of the 64-element slice
+    (513, 1000, 256, 3),   # N not a multiple of the tile, N % g != 0
+    (64, 72, 48, 2),       # a single, partial K slice
+    (200, 520, 96, 8),
+]
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("T,N,K,g", A16_SHAPES)
+def test_gemm_a16_matches_oracle(zq, bits, T, N, K, g):
+    if bits == 4 and K % 32:
+        pytest.skip("int4 needs K % 32 == 0")
+    _check_a16(zq, T, N, K, g, bits, seed=T + N + K)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("T,N,K", [(16, 256, 64), (300, 1000, 512), (1024, 768, 1024)])
+def test_gemm_a16_tiles(zq, bits, bn, T, N, K):
+    _check_a16(zq, T, N, K, 8, bits, seed=bn + T, bn=bn)
+
+
+def test_gemm_a16_persistent_loop_and_no_bias(zq):
+    """Three CTAs walk 36 tiles (two TMEM buffers and every pipeline slot
+    reused many times); no bias."""
+    _check_a16(zq, 600, 1536, 640, 12, 8, seed=5, bias=False, max_ctas=3)
+    _check_a16(zq, 600, 1536, 640, 12, 4, seed=6, bias=False, max_ctas=3)
+
+
+def test_gemm_a16_zero_scales_give_bias(zq):
+    T, N, K, g = 40, 256, 128, 4
+    X = synth.activations(T, K, seed=31)
+    b = synth.bias(N, 32)
+    q = np.zeros((N, K), np.int8)
+    sg = np.zeros(g, np.float32)
+    for bits, fn in ((8, zq.gemm_w8a16), (4, zq.gemm_w4a16)):
+        wdev = torch.from_numpy(oracle.pack_int4(q) if bits == 4 else q).cuda()
+        Y = fn(dev(X), wdev, torch.from_numpy(sg).cuda(), dev(b))
+        assert np.array_equal(host(Y).view(np.uint16),
+                              np.broadcast_to(b.numpy(), (T, N)).view(np.uint16))
+
+
+def test_gemm_a16_zero_tokens_is_a_no_op(zq):
+    X = torch.empty((0, 64), dtype=torch.float16, device="cuda")
+    q = torch.zeros((256, 64), dtype=torch.int8, device="cuda")
+    Y = zq.gemm_w8a16(X, q, torch.ones(4, device="cuda"))
+    assert Y.shape == (0, 256)
+
+
+A16_FULL = [("neox20b", 0, 4096, 8), ("neox20b", 0, 16, 8), ("gpt350m", 2, 16384, 4),
+            ("gptj6b", 3, 512, 4)]
+
+
+@pytest.mark.parametrize("layer,gi,T,bits", A16_FULL)
+def test_gemm_a16_full_size_sampled_rows(zq, layer, gi, T, bits):
+    """Full-size layers with FP16 activations (GPT-NeoX's attention input, the
+    W4/8A16 FFN weights); the oracle recomputes sampled token rows."""
+    inp = synth.gemm_inputs(layer, gi, T)
+    s = inp.spec
+    wq, sg = oracle.quantize_weights_groupwise(inp.W.numpy(), s.g, bits)
+    wdev = torch.from_numpy(oracle.pack_int4(wq) if bits == 4 else wq).cuda()
+    acc_d = torch.empty((T, s.N), dtype=torch.float32, device="cuda")
+    fn = zq.gemm_w4a16 if bits == 4 else zq.gemm_w8a16
+    Y = fn(dev(inp.X), wdev, torch.from_numpy(sg).cuda(), dev(inp.b), acc_dbg=acc_d)
+    rows = _sample_rows(T)[:6]
+    Xs = inp.X.numpy()[rows]
+    acc_ref, y_ref, Y_ref = oracle.gemm_a16(Xs, wq, sg, inp.b.numpy())
+    _assert_a16_close(Xs, wq, sg, host(acc_d)[rows], host(Y)[rows], acc_ref, y_ref, Y_ref)
+
+
 # ------------------------------------------------------------ errors on the device
 
 def test_bounded_wait_reports_timeout(zq):

@@ -42,6 +42,9 @@ MUTATIONS = {
                            "xmax = (1.0f - momentum) * xmax + momentum * bmax;"),
     "static_range_max_only": ("*A = fmaxf(fabsf(xmax), fabsf(xmin));", "*A = fabsf(xmax);"),
     "act_gelu_skipped": ("act == 1 ? d2h(zqo_gelu((double)v)) : f2h(v)", "act == 1 ? f2h(v) : f2h(v)"),
+    "a16_weights_transposed": ("(double)q[(size_t)o * K + k];", "(double)q[(size_t)k * N + o];"),
+    "a16_bias_dropped": ("(bias ? (double)h2f(bias[o]) : 0.0);", "0.0;"),
+    "a16_group_by_token": ("sum * (double)s_grp[zqo_group_of(o, N, g)]", "sum * (double)s_grp[zqo_group_of(t % N, N, g)]"),
 }
 
 

@@ -538,3 +538,56 @@ def test_token_wise_beats_static_on_varying_token_ranges():
     assert np.median(es[small]) > 4 * np.median(et[small])
     print(f"median per-token relative error: token-wise {np.median(et):.4f}, static {np.median(es):.4f}; "
           f"small-range tokens: token-wise {np.median(et[small]):.4f}, static {np.median(es[small]):.4f}")
+
+
+# ---------------------------------------------------------------- R15: FP16 activations
+
+def test_a16_small_integers_are_exact():
+    """X (q S)^T + b with small-integer activations and power-of-two group
+    scales: every step is exact, so the oracle equals integer arithmetic done
+    independently here (a transposed operand, a wrong group or a lost bias
+    fails).  g does not divide N, so the group boundaries are uneven."""
+    rng = np.random.default_rng(21)
+    T, N, K, g = 5, 14, 24, 3
+    X = rng.integers(-8, 9, (T, K)).astype(np.float16)
+    q = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    S = np.array([0.5, 0.25, 2.0], np.float32)
+    b = rng.integers(-4, 5, N).astype(np.float16)
+    acc, y, Y = oracle.gemm_a16(X, q, S, b)
+    ref_acc = np.array([[sum(int(X[t, k]) * int(q[o, k]) for k in range(K)) for o in range(N)]
+                        for t in range(T)])
+    grp = np.array([(o * g) // N for o in range(N)])
+    ref_y = ref_acc * S[grp].astype(np.float64) + b.astype(np.float64)
+    assert np.array_equal(acc, ref_acc)
+    assert np.array_equal(y, ref_y)
+    assert np.array_equal(Y.view(np.uint16), ref_y.astype(np.float16).view(np.uint16))
+    acc0, y0, _ = oracle.gemm_a16(X, q, S)
+    assert np.array_equal(y0, ref_acc * S[grp].astype(np.float64))
+
+
+def test_a16_matches_float64_matmul():
+    """Random fp16 activations and codes against numpy's float64 matmul of the
+    dequantized weights: the two sums differ only by double rounding."""
+    rng = np.random.default_rng(22)
+    T, N, K, g = 7, 40, 96, 5
+    X = (rng.standard_normal((T, K)) * 2).astype(np.float16)
+    q = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    S = (rng.random(g) * 0.01 + 1e-3).astype(np.float32)
+    b = (rng.standard_normal(N) * 0.1).astype(np.float16)
+    _, y, Y = oracle.gemm_a16(X, q, S, b)
+    Wd = q.astype(np.float64) * S[np.arange(N) * g // N].astype(np.float64)[:, None]
+    ref = X.astype(np.float64) @ Wd.T + b.astype(np.float64)
+    mag = np.abs(X.astype(np.float64)) @ np.abs(Wd).T + np.abs(b.astype(np.float64))
+    assert np.all(np.abs(y - ref) <= 1e-12 * mag)
+    assert np.array_equal(Y.view(np.uint16), y.astype(np.float16).view(np.uint16))
+
+
+def test_a16_zero_group_scale_leaves_the_bias():
+    """A group whose scale is 0 (an all-zero weight group) outputs the bias."""
+    rng = np.random.default_rng(23)
+    X = rng.standard_normal((3, 32)).astype(np.float16)
+    q = rng.integers(-127, 128, (8, 32)).astype(np.int8)
+    S = np.array([0.0, 0.02], np.float32)
+    b = np.arange(8, dtype=np.float16)
+    _, _, Y = oracle.gemm_a16(X, q, S, b)
+    assert np.array_equal(Y[:, :4], np.broadcast_to(b[:4], (3, 4)))

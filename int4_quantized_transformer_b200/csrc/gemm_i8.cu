@@ -87,9 +87,22 @@ struct Cfg {
   // per-stage cost (waits, commits, the unpack handoff) is paid once per
   // 16 KB of packed weights instead of once per 8 KB.
   static constexpr int KPS = (DEEP && BN <= 128) ? 2 : 1;
+  // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
+  // 32-column loads never leave the allocation.
+  static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
+  static constexpr int BUF_COLS = ACC_STRIDE;  // TMEM columns per accumulator buffer
+  // INT4 weight streaming up to BN = 128: the widened weights are written to
+  // tensor memory and the MMA reads its A operand from there, so shared
+  // memory carries only the packed codes and the activation tiles (it is
+  // the bandwidth that bounds this path).  Their ring of slots sits in TMEM
+  // after the two accumulator buffers, KPS * 32 columns per slot.
+  static constexpr bool TMEM_A = DEEP && BN <= 128;
+  static constexpr int A_COL0 = 2 * BUF_COLS;
+  static constexpr int TMEM_A_SLOTS_RAW = (512 - 2 * BUF_COLS) / (32 * KPS);
+  static constexpr int TMEM_A_SLOTS = TMEM_A_SLOTS_RAW > 4 ? 4 : TMEM_A_SLOTS_RAW;
   static constexpr int A_SLICE = BM * BK;                          // one K slice of A
   static constexpr int B_SLICE = (PAIR ? BN / 2 : BN) * BK;        // one K slice of B
-  static constexpr int A_BYTES = A_SLICE * KPS;
+  static constexpr int A_BYTES = TMEM_A ? 0 : A_SLICE * KPS;  // shared-memory A per stage
   static constexpr int B_BYTES = B_SLICE * KPS;
   static constexpr int P_BYTES = W4 ? W_ROWS * (BK / 2) * KPS : 0;  // packed row = KPS * 64 bytes
   // Weight streaming is bound by how fast TMA copies are issued: one issuing
@@ -106,7 +119,8 @@ struct Cfg {
   static constexpr int FREE_BYTES =
       kSmemBudget - NUM_EPI_WARPS_C * STG_BYTES - 8 * EPI_COLS * 8;
   static constexpr int STAGE_BYTES = DEEP ? A_BYTES : A_BYTES + B_BYTES + P_BYTES;
-  static constexpr int STAGES_RAW = DEEP ? (KPS == 2 ? 2 : 4) : FREE_BYTES / STAGE_BYTES;
+  static constexpr int STAGES_RAW =
+      TMEM_A ? TMEM_A_SLOTS : (DEEP ? (KPS == 2 ? 2 : 4) : FREE_BYTES / STAGE_BYTES);
   static constexpr int STAGES_CAP = WROWS ? 12 : 8;
   static constexpr int STAGES_ANY = STAGES_RAW > STAGES_CAP ? STAGES_CAP : STAGES_RAW;
   // the producers fill the shallow ring only when there is no deep ring
@@ -116,11 +130,8 @@ struct Cfg {
   static constexpr int PSTAGES_ANY = PSTAGES_RAW > 16 ? 16 : PSTAGES_RAW;
   static constexpr int PSTAGES = DEEP ? PSTAGES_ANY & ~1 : PSTAGES_ANY;  // deep (packed) ring
   static constexpr int EPI_ARRIVALS = PAIR ? 2 * NUM_EPI_WARPS_C : NUM_EPI_WARPS_C;
-  // TMEM columns per accumulator buffer: at least 32 so that the epilogue's
-  // 32-column loads never leave the allocation.
-  static constexpr int ACC_STRIDE = BN < 32 ? 32 : BN;
-  static constexpr int BUF_COLS = ACC_STRIDE;  // TMEM columns per accumulator buffer
-  static constexpr int TMEM_COLS = pow2_at_least(2 * BUF_COLS);
+  static constexpr int TMEM_COLS =
+      pow2_at_least(2 * BUF_COLS + (TMEM_A ? STAGES * 32 * KPS : 0));
   static constexpr int NUM_EPI_WARPS = NUM_EPI_WARPS_C;
   static constexpr int NUM_UNPACK_WARPS = W4 ? 4 : 0;
   static constexpr int NUM_WARPS = 1 + NUM_PROD_WARPS + NUM_EPI_WARPS + NUM_UNPACK_WARPS;
@@ -146,6 +157,9 @@ struct Cfg {
                 "unpack steps keep the row's swizzle phase");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(TMEM_COLS <= 512, "TMEM accumulators");
+  static_assert(!TMEM_A || (KPS == 2 && STAGES >= 2 && P_BYTES == BM * 128 &&
+                            A_COL0 + STAGES * 32 * KPS <= TMEM_COLS),
+                "TMEM operand ring: packed rows of two K slices (128 bytes, 128B swizzle)");
   static_assert(EPI_COLS <= 128, "epilogue prefetch holds at most four columns per lane");
 };
 
@@ -455,10 +469,20 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           tc_fence_after();
 #pragma unroll
           for (int h = 0; h < C::KPS; ++h) {
-            const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES + h * C::A_SLICE));
             const uint64_t db = make_sw128_desc(
                 smem_u32(sB + (C::DEEP ? pst : stage) * C::B_BYTES + h * C::B_SLICE));
             const bool first = kb == t.kb0 && h == 0;  // the unit's first K slice
+            if constexpr (C::TMEM_A) {
+              // A from TMEM: K = 32 bytes = 8 columns per MMA
+              const uint32_t a_tm = tmem_base + static_cast<uint32_t>(
+                                                    C::A_COL0 + (stage * C::KPS + h) * 32);
+#pragma unroll
+              for (int k = 0; k < BK / UMMA_K; ++k)
+                mma_i8_ts(d_tmem, a_tm + static_cast<uint32_t>(8 * k),
+                          db + static_cast<uint64_t>(2 * k), idesc, (!first || k > 0) ? 1u : 0u);
+              continue;
+            }
+            const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES + h * C::A_SLICE));
 #pragma unroll
             for (int k = 0; k < BK / UMMA_K; ++k) {
               // advance the start address by k*32 bytes (>>4 = 2k) inside the swizzle row
@@ -770,6 +794,44 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
                                 p.status, 5)) {
             ok = false;
             break;
+          }
+          if constexpr (C::TMEM_A) {
+            // Lane = weight row r of the tile, in this warp's TMEM lane
+            // quadrant.  Its packed row (two K slices, 128 bytes, landed by
+            // TMA in the 128B-swizzled layout: 16-byte chunk c of row r at
+            // c ^ (r % 8)) is widened to codes*16 and written to the ring
+            // slot's 2 x 32 TMEM columns (four k per column, in k order).
+            const int r = (warp & 3) * 32 + lane;
+            const uint8_t* prow = sP + pst * C::P_BYTES + r * PROW;
+            const uint32_t a_tm = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
+                                  static_cast<uint32_t>(C::A_COL0 + stage * C::KPS * 32);
+#pragma unroll
+            for (int h = 0; h < C::KPS; ++h) {
+              uint32_t w[32];
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const uint4 v =
+                    *reinterpret_cast<const uint4*>(prow + (((h * 4 + c) ^ (r & 7)) << 4));
+                unpack8_x16(v.x, w[8 * c], w[8 * c + 1]);
+                unpack8_x16(v.y, w[8 * c + 2], w[8 * c + 3]);
+                unpack8_x16(v.z, w[8 * c + 4], w[8 * c + 5]);
+                unpack8_x16(v.w, w[8 * c + 6], w[8 * c + 7]);
+              }
+              tmem_st_32x32b_x32(a_tm + static_cast<uint32_t>(h * 32), w);
+            }
+            tmem_st_wait();
+            tc_fence_before();  // the stores are ordered before the MMA warp's reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ready_bar[stage]);
+            if (++pst == C::PSTAGES) {
+              pst = 0;
+              pphase ^= 1;
+            }
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
           }
           // Thread ut handles 16-byte output chunk j = ut % 8 of rows
           // r = ut / 8 + UROWS i: stepping a multiple of 8 rows keeps r % 8,
@@ -1168,9 +1230,13 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
                      CU_TENSOR_MAP_SWIZZLE_128B))
     return ZQ_ERR_CUDA;
   if (w4) {
-    // one box per stage: plan.kps K slices of 64 packed bytes per row
+    // one box per stage: plan.kps K slices of 64 packed bytes per row; with
+    // the TMEM operand ring (weight rows, BN <= 128) each thread reads a
+    // whole 128-byte row, so those rows land 128B-swizzled (conflict-free)
+    const bool tmem_a = plan.wrows && plan.bn <= 128;
     if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K / 2, N, K / 2,
-                       plan.kps * (BK / 2), w_rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+                       plan.kps * (BK / 2), w_rows,
+                       tmem_a ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
       return ZQ_ERR_CUDA;
   } else {
     if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, BK, w_rows,

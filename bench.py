@@ -57,7 +57,7 @@ def load_peaks():
 NCU_TRAFFIC = {
     # profiles/gemm_i8_dram_traffic.md, bert_base ffn1 row (the fp16 output
     # is still in L2 when the kernel ends, so DRAM writes read 0)
-    ("ffn1", 768, 3072, 4096): {"bytes": 5576448 + 0, "source": "b6c00368f02b"},
+    ("ffn1", 768, 3072, 4096): {"bytes": 5571328 + 0, "source": "1c18476bf6fe"},
 }
 
 
@@ -162,8 +162,8 @@ class LayerStep:
             s = gi.spec
             W = gi.W.to(device)
             Wq, sg = zq.quantize_weights_groupwise(W, s.g, s.bits)
-            del W
             it = {
+                "W16": W,  # the fp16 weights, for the fp16 cuBLAS comparison only
                 "spec": s,
                 "X": gi.X.to(device),
                 "gamma": None if gi.gamma is None else gi.gamma.to(device),
@@ -345,6 +345,25 @@ def gpu_arm(args, dist_on, rank, world):
                 tot, _ = time_steps(fn, reps, flush_buf, stream)
                 kern[(s.name, kind)] = tot / reps
         kern_method = f"eager launches after an L2 flush ({type(exc).__name__})"
+    # ---- the same shapes in fp16 through cuBLAS (torch.addmm: X W^T + b),
+    # and cuBLAS's own INT8 GEMM (torch._int_mm, int32 out, no scales) on the
+    # dominant shape: library references, timed the same way
+    ref16 = {}
+    ref_i8 = None
+    ref16_error = None
+    try:
+        for it in step.items:
+            fn16 = lambda it=it: torch.addmm(it["b"], it["X"], it["W16"].t())
+            fn16()  # cuBLAS sets up its handle and workspace outside the capture
+            torch.cuda.synchronize()
+            ref16[it["spec"].name] = max(time_graph(graph_of(fn16)) - base_ms, 1e-6) / reps
+        ref16_step_ms, _ = time_steps(lambda: [torch.addmm(it["b"], it["X"], it["W16"].t())
+                                               for it in step.items],
+                                      max(3, args.steps // 2), flush_buf, stream)
+        ref16_step_ms /= max(3, args.steps // 2)
+    except Exception as exc:
+        ref16, ref16_step_ms = {}, None
+        ref16_error = f"{type(exc).__name__}: {exc}"
     gemm_ms = sum(v for (n, k), v in kern.items() if k == "gemm")
     ln_ms = sum(v for (n, k), v in kern.items() if k == "ln")
     peak_tops = INT8_PER_BF16 * float(peaks["bf16_tflops"])
@@ -354,6 +373,17 @@ def gpu_arm(args, dist_on, rank, world):
     dom_ms = kern[(dom_spec.name, "gemm")]
     dom_ops = 2.0 * T * dom_spec.N * dom_spec.K
     achieved_tops = dom_ops / (dom_ms * 1e-3) / 1e12
+    if T > 16:
+        try:
+            x8 = torch.randint(-127, 128, (T, dom_spec.K), dtype=torch.int8, device=device)
+            w8 = torch.randint(-127, 128, (dom_spec.N, dom_spec.K), dtype=torch.int8, device=device)
+            torch._int_mm(x8, w8.t())
+            torch.cuda.synchronize()
+            ref_i8 = max(time_graph(graph_of(lambda: torch._int_mm(x8, w8.t()))) - base_ms,
+                         1e-6) / reps
+            del x8, w8
+        except Exception:
+            ref_i8 = None
     all_gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
 
     # ---- end to end through the C ABI: pinned host inputs in, outputs out
@@ -419,6 +449,16 @@ def gpu_arm(args, dist_on, rank, world):
             "kernel_time_method": kern_method,
         },
         "kernels_us": {f"{n}.{k}": round(v * 1e3, 2) for (n, k), v in kern.items()},
+        "fp16_cublas": {"error": ref16_error} if not ref16 else {
+            "what": "torch.addmm(bias, X, W^T) in fp16 (cuBLAS) on each GEMM shape of the step, "
+                    "timed as the kernels above; step = the four GEMMs back to back (no LayerNorm)",
+            "gemm_us": {n: round(v * 1e3, 2) for n, v in ref16.items()},
+            "step_us": None if ref16_step_ms is None else round(ref16_step_ms * 1e3, 2),
+            "gemm_speedup": round(sum(ref16.values()) / gemm_ms, 3),
+            "step_speedup": None if ref16_step_ms is None else round(ref16_step_ms / ms_per_step, 3),
+            "dominant_fp16_tflops": round(dom_ops / (ref16[dom_spec.name] * 1e-3) / 1e12, 1),
+            "dominant_cublas_int8_us": None if ref_i8 is None else round(ref_i8 * 1e3, 2),
+        },
         "ln_quant_gbs": round(sum(3 * it["T"] * it["spec"].K for it in step.items) / (ln_ms * 1e-3) / 1e9, 1),
         "offline_wquant_ms": round(wquant_s * 1e3, 2),
         "e2e": {"value": round(whole_job_tops(ops, world, e2e_ms), 2), "unit": "TOPS",

@@ -515,9 +515,19 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   if (!aligned16(X) || !aligned16(Wq) || !aligned16(Y) || (bias && !aligned16(bias)) ||
       (acc_dbg && !aligned16(acc_dbg)))
     return ZQ_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // A handful of tokens: the CUDA-core matrix-vector path (the 128-row token
+  // tile would leave the tensor cores nearly idle while the weights stream).
+  const int forced_path = option(ZQ_OPT_GEMM_PATH);
+  if (forced_path == 3 || (forced_path == 0 && T <= kGemvMaxTokens)) {
+    if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
+    return launch_gemv_a16(w4 ? 4 : 8, X, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg,
+                           option(ZQ_OPT_MAX_CTAS), st) == cudaSuccess
+               ? ZQ_OK
+               : ZQ_ERR_CUDA;
+  }
   const int fbn = option(ZQ_OPT_GEMM_BN);
   if (fbn && fbn != 128 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int sms = num_sms();
   const A16Plan plan = plan_a16(T, N, K, sms, fbn);
 

@@ -190,10 +190,16 @@ def test_gemm_a16_argument_rules(zq):
     assert L.zq_gemm_w4a16(FAKE, FAKE, FAKE, 4, None, 16, 256, 48, FAKE, None, None) == zq.ZQ_ERR_SHAPE
     # no tokens: nothing to check, nothing launched
     assert L.zq_gemm_w8a16(None, None, None, 4, None, 0, 256, 64, None, None, None) == zq.ZQ_OK
+    # the matrix-vector path takes at most four tokens
+    with zq.options(path=3):
+        assert L.zq_gemm_w8a16(FAKE, FAKE, FAKE, 4, None, 5, 256, 64, FAKE, None,
+                               None) == zq.ZQ_ERR_UNSUPPORTED
     # only the 128- and 256-wide tiles exist for FP16 activations
     with zq.options(bn=192):
         assert L.zq_gemm_w8a16(FAKE, FAKE, FAKE, 4, None, 16, 256, 64, FAKE, None,
                                None) == zq.ZQ_ERR_UNSUPPORTED
+        # (a T <= 4 call takes the matrix-vector path, where the tile width
+        # does not apply: it is not checked here because it would launch)
 
 
 def test_w4a8_needs_k_multiple_of_32(zq):

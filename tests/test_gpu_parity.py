@@ -471,6 +471,23 @@ def test_gemm_a16_tiles(zq, bits, bn, T, N, K):
     _check_a16(zq, T, N, K, 8, bits, seed=bn + T, bn=bn)
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+@pytest.mark.parametrize("N,K,g", [(256, 64, 4), (1000, 4160, 5), (8, 96, 1), (4104, 3072, 24)])
+def test_gemm_a16_gemv_path(zq, bits, T, N, K, g):
+    """T <= 4 runs on the CUDA-core matrix-vector kernel (automatic and forced)."""
+    if bits == 4 and K % 32:
+        pytest.skip("int4 needs K % 32 == 0")
+    _check_a16(zq, T, N, K, g, bits, seed=T * 7 + N)
+    _check_a16(zq, T, N, K, g, bits, seed=T * 7 + N + 1, bias=False, path=3, max_ctas=5)
+
+
+def test_gemm_a16_small_t_on_tensor_cores(zq):
+    """The tensor-core path forced for a few tokens (one partial 128-row tile)."""
+    _check_a16(zq, 3, 520, 256, 8, 8, seed=41, path=1)
+    _check_a16(zq, 1, 520, 256, 8, 4, seed=42, path=1)
+
+
 def test_gemm_a16_persistent_loop_and_no_bias(zq):
     """Three CTAs walk 36 tiles (two TMEM buffers and every pipeline slot
     reused many times); no bias."""
@@ -498,7 +515,8 @@ def test_gemm_a16_zero_tokens_is_a_no_op(zq):
     assert Y.shape == (0, 256)
 
 
-A16_FULL = [("neox20b", 0, 4096, 8), ("neox20b", 0, 16, 8), ("gpt350m", 2, 16384, 4),
+A16_FULL = [("neox20b", 0, 4096, 8), ("neox20b", 0, 16, 8), ("neox20b", 2, 1, 4), ("gptj6b", 0, 4, 8),
+            ("gpt350m", 2, 16384, 4),
             ("gptj6b", 3, 512, 4)]
 
 

@@ -519,8 +519,8 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   // A handful of tokens: the CUDA-core matrix-vector path (the 128-row token
   // tile would leave the tensor cores nearly idle while the weights stream).
   const int forced_path = option(ZQ_OPT_GEMM_PATH);
-  if (forced_path == 3 || (forced_path == 0 && T <= kGemvMaxTokens)) {
-    if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
+  if (forced_path == 3 || (forced_path == 0 && T <= kGemvA16MaxTokens)) {
+    if (T > kGemvA16MaxTokens) return ZQ_ERR_UNSUPPORTED;
     return launch_gemv_a16(w4 ? 4 : 8, X, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg,
                            option(ZQ_OPT_MAX_CTAS), st) == cudaSuccess
                ? ZQ_OK

@@ -238,7 +238,7 @@ cudaError_t launch_a16_tt(const void* X, const void* W, const float* s_grp, int 
 cudaError_t launch_gemv_a16(int bits, const void* X, const void* W, const float* s_grp, int g,
                             const void* bias, int T, int N, int K, void* Y, float* acc_dbg,
                             int max_ctas, cudaStream_t st) {
-  if (T < 1 || T > kGemvMaxTokens) return cudaErrorInvalidValue;
+  if (T < 1 || T > kGemvA16MaxTokens) return cudaErrorInvalidValue;
   if (bits == 4) {
     if (T == 1) return launch_a16_tt<4, 1>(X, W, s_grp, g, bias, T, N, K, Y, acc_dbg, max_ctas, st);
     if (T == 2) return launch_a16_tt<4, 2>(X, W, s_grp, g, bias, T, N, K, Y, acc_dbg, max_ctas, st);

@@ -27,7 +27,8 @@ cudaError_t launch_gemv_i8(int bits, const int8_t* Xq, const float* s_tok, const
                            const float* s_grp, int g, const void* bias, int T, int N, int K,
                            void* Y, int32_t* acc_dbg, int max_ctas, cudaStream_t st);
 // The CUDA-core matrix-vector path of the FP16-activation layer (gemv_a16.cu),
-// for at most kGemvMaxTokens tokens: bits = 4 (packed INT4) or 8.
+// for at most kGemvA16MaxTokens tokens: bits = 4 (packed INT4) or 8.
+constexpr int kGemvA16MaxTokens = 4;
 cudaError_t launch_gemv_a16(int bits, const void* X, const void* W, const float* s_grp, int g,
                             const void* bias, int T, int N, int K, void* Y, float* acc_dbg,
                             int max_ctas, cudaStream_t st);

@@ -159,7 +159,9 @@ zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
  * zq_gemm_w4a8 -- as zq_gemm_w8a8 with INT4 weights (Sec. 3.4 "Which weights
  * get INT4": FFN weights in INT4).  Wq4 is uint8 [N][K/2] in the layout of
  * zq_quantize_weights_groupwise(bits=4); the kernel unpacks the nibbles to
- * int8 in shared memory before each tensor-core MMA.
+ * int8 before each tensor-core MMA: in shared memory for token-row tiles,
+ * in tensor memory (the MMA's A operand) for weight-row tiles, which this
+ * function uses up to T = 128 and for T >= 1024 when K >= 2048.
  * Requirements as zq_gemm_w8a8, plus K % 32 == 0 and K <= 132096.
  */
 zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,

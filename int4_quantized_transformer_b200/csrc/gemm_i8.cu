@@ -989,6 +989,20 @@ int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b
 // Largest token count the automatic choice sends to the matrix-vector path.
 int gemv_max_tokens(bool w4) { return w4 ? kGemvMaxTokens : 2; }
 
+// The automatic choice of weight rows on the MMA M side (above the
+// matrix-vector range).  INT8 weights: up to 256 tokens (weight streaming).
+// INT4 weights: up to 128 tokens, and also for prefill-sized token counts
+// with long rows (T >= 1024, K >= 2048), where widening the weights into
+// tensor memory beats the token-row tiles' widening through shared memory
+// (measured on B200: GPT-NeoX FFN1/FFN2 at T = 4096 697/767 us instead of
+// 772/873 us, GPT-3 350M FFN2 at T = 16384 87 us instead of 117 us); with
+// short rows (K = 1024) or few tokens the token-row tiles stay ahead, since
+// each weight-row tile re-reads its whole activation block.
+bool use_weight_rows(int T, int K, bool w4) {
+  if (!w4) return T <= 256;
+  return T <= 128 || (T >= 1024 && K >= 2048);
+}
+
 // fp16 output [T][N]: 32 x 32 boxes written by the epilogue warps
 bool encode_y_map(CUtensorMap* my, void* Y, int T, int N) {
   return encode_tma_2d(my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
@@ -1004,8 +1018,11 @@ Plan plan_wrows(int T, int N, int K, int sms, int forced_split, bool w4) {
   Plan p{};
   p.wrows = true;
   p.pair = false;
+  // INT4 weights: at most 128 tokens per tile, so that the widened weights
+  // can live in tensor memory next to the two accumulator buffers
+  const int bn_cap = w4 ? 128 : 256;
   int bn = 16;
-  while (bn < T && bn < 256) bn *= 2;
+  while (bn < T && bn < bn_cap) bn *= 2;
   p.bn = bn;
   const int kps = (w4 && bn <= 128) ? 2 : 1;
   p.kps = kps;
@@ -1170,7 +1187,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
                : ZQ_ERR_CUDA;
   }
   Plan plan;
-  if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
+  if (forced_path == 2 || (forced_path == 0 && use_weight_rows(T, K, w4))) {
     plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K), w4);
   } else {
     const int fbn = option(ZQ_OPT_GEMM_BN);

@@ -185,6 +185,16 @@ def test_gemm_auto(zq, bits, T, N, K, g):
     _check_gemm(zq, T, N, K, g, bits, seed=T + N + K)
 
 
+@pytest.mark.parametrize("T,N,K,g", [(1100, 640, 2048, 5), (130, 512, 2048, 8), (128, 384, 4096, 3),
+                                     (2048, 256, 3072, 4), (1024, 1024, 1024, 16)])
+def test_gemm_w4_tiling_choices(zq, T, N, K, g):
+    """INT4 weights choose weight-row tiles (widened weights in TMEM) up to
+    T = 128 and for T >= 1024 with K >= 2048, token-row tiles otherwise; both
+    sides of each boundary, and the forced alternative, match the oracle."""
+    _check_gemm(zq, T, N, K, g, 4, seed=T + K)
+    _check_gemm(zq, T, N, K, g, 4, seed=T + K + 1, path=2)
+
+
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("bn", [128, 192, 256])
 @pytest.mark.parametrize("T,N,K", [(16, 256, 64), (300, 1000, 512), (1024, 768, 1024)])

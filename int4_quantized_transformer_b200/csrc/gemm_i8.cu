@@ -173,6 +173,9 @@ struct GemmParams {
   int* status;
   int T, N, K, g;
   int m_tiles, n_tiles, k_blocks, splits, kb_per_split, num_units;
+  // unit order: 0 = M tiles fastest (consecutive units, which run at the
+  // same time, share their N-side operand tile), 1 = N tiles fastest
+  int n_fastest;
 };
 
 struct Unit {
@@ -183,8 +186,13 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmParams& p) {
   Unit r;
   const int split = u % p.splits;
   const int rest = u / p.splits;
-  r.m = rest % p.m_tiles;
-  r.n = rest / p.m_tiles;
+  if (p.n_fastest) {
+    r.n = rest % p.n_tiles;
+    r.m = rest / p.n_tiles;
+  } else {
+    r.m = rest % p.m_tiles;
+    r.n = rest / p.m_tiles;
+  }
   r.kb0 = split * p.kb_per_split;
   r.kb1 = min(p.k_blocks, r.kb0 + p.kb_per_split);
   return r;
@@ -1230,6 +1238,11 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   gp.splits = plan.splits;
   gp.kb_per_split = plan.kb_per_split;
   gp.num_units = plan.units;
+  // Weight rows with several token tiles: when the weights are the larger
+  // operand, let the CTAs running at the same time share a weight tile (each
+  // weight tile then comes from DRAM once, the activations from L2).
+  gp.n_fastest = plan.wrows && plan.n_tiles > 1 &&
+                 static_cast<double>(N) * K * (w4 ? 0.5 : 1.0) > static_cast<double>(T) * K;
   if (plan.wrows && plan.splits > 1) {
     Workspace* w = nullptr;
     if (ensure_workspace(static_cast<size_t>(plan.splits) * T * N, &w) != cudaSuccess)
@@ -1396,6 +1409,8 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   gp.splits = plan.splits;
   gp.kb_per_split = plan.kb_per_split;
   gp.num_units = plan.units;
+  gp.n_fastest = plan.wrows && plan.n_tiles > 1 &&
+                 static_cast<double>(N) * K > static_cast<double>(T) * K;
   if (plan.wrows && plan.splits > 1) {
     const size_t partial = static_cast<size_t>(plan.splits) * T * N;
     if (partial > kNoAllocPartialInts) return ZQ_ERR_SHAPE;

@@ -423,6 +423,8 @@ def gpu_arm(args, dist_on, rank, world):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5),
+        "ms_per_step_median": round(statistics.median(per_step), 5),
+        "ms_per_step_best": round(min(per_step), 5),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -502,6 +504,17 @@ def prepare_oracle(layer, T):
     return inputs
 
 
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(layer, T, rows):
     rows = min(rows, T)
     inputs = prepare_oracle(layer, T)
@@ -510,6 +523,7 @@ def cpu_baseline(layer, T, rows):
     dt = time.perf_counter() - t0
     ops = gemm_ops([gi.spec for gi in inputs], rows)
     return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "host_cpu_model": host_cpu_model(),
             "sample": f"{rows} of {T} tokens of every GEMM of the step (LN+quant, exact int GEMM, "
                       f"dequant), single-threaded plain C, {dt:.1f} s",
             "host_cpus": os.cpu_count()}
@@ -540,7 +554,8 @@ def reference_arm(args, rank, world):
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": f"{layer} layer, T={T} tokens (oracle timed on a {rows}-token sample)",
                    "tokens": T},
-        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": 1, "kind": "oracle", "sample": sample,
+                         "host_cpu_model": host_cpu_model(), "host_cpus": os.cpu_count()},
         "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

@@ -44,7 +44,9 @@ def main():
     ap.add_argument("--bn", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--pair", type=int, default=0, help="1 = single-CTA tiles, 2 = CTA pairs")
-    ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
+    ap.add_argument("--eager", action="store_true",
+                    help="eager launches instead of a graph (for ncu captures: the printed time then "
+                         "includes host launch latency)")
     ap.add_argument("--flush", action="store_true",
                     help="flush the L2 before every launch (512 MB write + 256 MB read, as in bench.py)")
     a = ap.parse_args()

@@ -187,7 +187,8 @@ zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
  * Runs on tcgen05 tensor cores (kind::f16), except for T <= 4: a
  * memory-bound matrix-vector product on CUDA cores (exact products, fp32
  * fma sums).  ZQ_OPT_GEMM_PATH = 3 forces that path (T <= 4), 1 or 2 the
- * tensor cores.
+ * tensor cores; ZQ_OPT_CTA_PAIR = 2 forces 256-row units shared by a CTA
+ * pair (measured slower, never chosen automatically).
  * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
  * 16 <= K <= 2^20, K % 16 == 0, 1 <= g <= N, pointers 16-byte aligned.
  * Errors: as zq_gemm_w8a8 (argument errors before any launch).

@@ -55,14 +55,19 @@ constexpr int tmem_cols_for(int v) {
   return p;
 }
 
-template <int BN_, bool W4_>
+template <int BN_, bool W4_, bool PAIR_>
 struct A16Cfg {
   static constexpr int BN = BN_;
   static constexpr bool W4 = W4_;
+  // CTA pair (cta_group::2): a 256 x BN tile per pair; each CTA holds 128
+  // token rows of A, widens BN/2 weight rows of B, and keeps 128 rows of D.
+  static constexpr bool PAIR = PAIR_;
+  static constexpr int TILE_M = PAIR ? 2 * kBM : kBM;  // token rows of a unit
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;    // weight rows this CTA widens
   static constexpr int A_BYTES = kBM * 128;            // fp16 activations of one slice
-  static constexpr int B_BYTES = BN * 128;             // widened weights of one slice
+  static constexpr int B_BYTES = B_ROWS * 128;         // widened weights of one slice
   static constexpr int CODE_ROW = W4 ? kKE / 2 : kKE;  // code bytes per weight row and slice
-  static constexpr int P_BYTES = BN * CODE_ROW;        // codes as stored in memory
+  static constexpr int P_BYTES = B_ROWS * CODE_ROW;    // codes as stored in memory
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
   static constexpr int EPI_COLS = BN / 2;              // columns of one epilogue warp
   static constexpr int STG_BYTES = 32 * 32 * 2;        // one 32 x 32 fp16 output block
@@ -80,12 +85,14 @@ struct A16Cfg {
   static constexpr int EPI_BYTES = kEpiWarps * EPI_COLS * 2 * 4;
   static constexpr int OFF_STG = ((OFF_EPI + EPI_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_BAR = OFF_STG + kEpiWarps * STG_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 4 + 1;
+  static constexpr int NUM_BARS = 4 * STAGES + 4 + 1;
+  static constexpr int READY_ARRIVALS = PAIR ? 2 * kCvtWarps : kCvtWarps;
+  static constexpr int EPI_ARRIVALS = PAIR ? 2 * kEpiWarps : kEpiWarps;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(STAGES >= 2, "not enough shared memory for two stages");
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "MMA N and the epilogue's 64-column steps");
-  static_assert(BN % 16 == 0, "widening steps of 16 rows keep each row's swizzle phase");
+  static_assert(B_ROWS % 16 == 0, "widening steps of 16 rows keep each row's swizzle phase");
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(P_BYTES % 128 == 0, "TMA destination alignment");
   static_assert(EPI_COLS <= 128, "epilogue prefetch holds at most four columns per lane");
@@ -167,10 +174,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   float* sEpi = reinterpret_cast<float*>(smem + C::OFF_EPI);
   uint8_t* sStg = smem + C::OFF_STG;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full_bar = bars;                  // [STAGES] activations + codes landed
-  uint64_t* ready_bar = bars + STAGES;        // [STAGES] widened weights written
+  // Single CTA: full = activations + codes landed.  Pair: full (the leader's)
+  // counts both CTAs' activation tiles, pfull this CTA's codes.
+  uint64_t* full_bar = bars;                  // [STAGES]
+  uint64_t* ready_bar = bars + STAGES;        // [STAGES] widened weights written (leader's, pair)
   uint64_t* empty_bar = bars + 2 * STAGES;    // [STAGES] the MMAs reading the stage are done
-  uint64_t* tfull_bar = bars + 3 * STAGES;    // [2] accumulator buffer complete
+  uint64_t* pfull_bar = bars + 3 * STAGES;    // [STAGES] pair: this CTA's codes landed
+  uint64_t* tfull_bar = bars + 4 * STAGES;    // [2] accumulator buffer complete
   uint64_t* tempty_bar = tfull_bar + 2;       // [2] accumulator buffer drained
   uint64_t* drain_bar = tempty_bar + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -178,18 +188,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x & 31;
-  const int unit0 = static_cast<int>(blockIdx.x);
-  const int ustep = static_cast<int>(gridDim.x);
+  // a pair works on one unit at a time; crank 0 (the leader) issues the MMAs
+  const uint32_t crank = C::PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = C::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ustep = C::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&ready_bar[s], kCvtWarps);
+      mbar_init(&ready_bar[s], C::READY_ARRIVALS);
       mbar_init(&empty_bar[s], 1);
+      mbar_init(&pfull_bar[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], kEpiWarps);
+      mbar_init(&tempty_bar[b], C::EPI_ARRIVALS);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -199,11 +212,17 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     tma_prefetch_desc(&map_y);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (C::PAIR) {
+      tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   // Nothing above touches global memory; what follows may read what the
@@ -224,16 +243,30 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ok = true;
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const int m = u % p.m_tiles, n = u / p.m_tiles;
+        const int act_row = m * C::TILE_M + static_cast<int>(crank) * kBM;
+        const int w_row = n * BN + static_cast<int>(crank) * C::B_ROWS;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.status, 21)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full_bar[stage], bytes);
           // slices past K (and rows past T or N) read the TMA's zero fill
-          tma_load_2d(sA + stage * C::A_BYTES, &map_x, &full_bar[stage], kb * kKE, m * kBM, pol_x);
-          tma_load_2d(sP + stage * C::P_BYTES, &map_w, &full_bar[stage], kb * C::CODE_ROW, n * BN,
-                      pol_w);
+          if constexpr (C::PAIR) {
+            // both CTAs' activation tiles complete on the leader's full
+            // barrier (the MMA reads them); this CTA's codes on its own
+            // pfull barrier (its widening warps read them)
+            if (crank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2u * C::A_BYTES);
+            tma_load_2d_pair(sA + stage * C::A_BYTES, &map_x,
+                             mapa_shared(smem_u32(&full_bar[stage]), 0), kb * kKE, act_row, pol_x);
+            mbar_arrive_expect_tx(&pfull_bar[stage], static_cast<uint32_t>(C::P_BYTES));
+            tma_load_2d(sP + stage * C::P_BYTES, &map_w, &pfull_bar[stage], kb * C::CODE_ROW, w_row,
+                        pol_w);
+          } else {
+            mbar_arrive_expect_tx(&full_bar[stage], bytes);
+            tma_load_2d(sA + stage * C::A_BYTES, &map_x, &full_bar[stage], kb * kKE, act_row, pol_x);
+            tma_load_2d(sP + stage * C::P_BYTES, &map_w, &full_bar[stage], kb * C::CODE_ROW, w_row,
+                        pol_w);
+          }
           ++fills[stage];
           if (++stage == STAGES) {
             stage = 0;
@@ -241,15 +274,21 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           }
         }
       }
-      // every copy issued lands before the CTA may exit
+      // every copy issued lands before the CTA may exit (for a pair, the
+      // leader's full barriers count both CTAs' activation copies; the
+      // follower exits only after the final cluster barrier)
       int no_abort = 0;
-      for (int s = 0; s < STAGES; ++s)
-        if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 22);
+      if (!C::PAIR || crank == 0)
+        for (int s = 0; s < STAGES; ++s)
+          if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 22);
+      if (C::PAIR)
+        for (int s = 0; s < STAGES; ++s)
+          if (fills[s]) mbar_wait(&pfull_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 28);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_f16(kBM, BN);
+    if (lane == 0 && (!C::PAIR || crank == 0)) {
+      constexpr uint32_t idesc = make_idesc_f16(C::TILE_M, BN);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -260,8 +299,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          // the widening warps arrive only after the stage's copies landed
-          if (!mbar_wait(&ready_bar[stage], phase, abort_flag, p.status, 24)) {
+          // the widening warps arrive only after the stage's codes landed
+          // (single CTA: with the activations, on the same barrier); a pair
+          // also waits for both CTAs' activation tiles
+          if (!mbar_wait(&ready_bar[stage], phase, abort_flag, p.status, 24) ||
+              (C::PAIR && !mbar_wait(&full_bar[stage], phase, abort_flag, p.status, 29))) {
             ok = false;
             break;
           }
@@ -269,24 +311,38 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           const uint64_t da = make_sw128_desc(smem_u32(sA + stage * C::A_BYTES));
           const uint64_t db = make_sw128_desc(smem_u32(sB + stage * C::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < kKE / kUmmaK; ++k)  // start address + k*32 bytes (>>4 = 2k)
-            mma_f16(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
-                    idesc, (kb > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&empty_bar[stage]);
+          for (int k = 0; k < kKE / kUmmaK; ++k) {  // start address + k*32 bytes (>>4 = 2k)
+            if constexpr (C::PAIR)
+              mma_f16_pair(d_tmem, da + static_cast<uint64_t>(2 * k),
+                           db + static_cast<uint64_t>(2 * k), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            else
+              mma_f16(d_tmem, da + static_cast<uint64_t>(2 * k), db + static_cast<uint64_t>(2 * k),
+                      idesc, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          if constexpr (C::PAIR)
+            mma_commit_pair_mc(&empty_bar[stage], 0x3);
+          else
+            mma_commit(&empty_bar[stage]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        mma_commit(&tfull_bar[buf]);
+        if constexpr (C::PAIR)
+          mma_commit_pair_mc(&tfull_bar[buf], 0x3);
+        else
+          mma_commit(&tfull_bar[buf]);
         if (++buf == 2) {
           buf = 0;
           tphase ^= 1;
         }
       }
       // every MMA issued completes before TMEM is released
-      mma_commit(drain_bar);
+      if constexpr (C::PAIR)
+        mma_commit_pair_mc(drain_bar, 0x1);
+      else
+        mma_commit(drain_bar);
       int no_abort = 0;
       mbar_wait(drain_bar, 0, &no_abort, p.status, 25);
     }
@@ -337,8 +393,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       if (!a16_wait_warp(&tfull_bar[buf], tphase, abort_flag, p.status, 26)) break;
       tc_fence_after();
       fetch(u + ustep);
-      const int tok = m * kBM + row_in_tile;
-      const int row0 = m * kBM + quad * 32;
+      const int tok = m * C::TILE_M + static_cast<int>(crank) * kBM + row_in_tile;
+      const int row0 = m * C::TILE_M + static_cast<int>(crank) * kBM + quad * 32;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf * BN);
 
@@ -396,7 +452,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+      if (lane == 0) {
+        if constexpr (C::PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tempty_bar[buf]), 0));
+        else
+          mbar_arrive(&tempty_bar[buf]);
+      }
       if (++buf == 2) {
         buf = 0;
         tphase ^= 1;
@@ -417,14 +478,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
     bool ok = true;
     for (int u = unit0; ok && u < p.num_units; u += ustep) {
       for (int kb = 0; kb < p.k_blocks; ++kb) {
-        if (!a16_wait_warp(&full_bar[stage], phase, abort_flag, p.status, 27)) {
+        if (!a16_wait_warp(C::PAIR ? &pfull_bar[stage] : &full_bar[stage], phase, abort_flag,
+                           p.status, 27)) {
           ok = false;
           break;
         }
         const uint8_t* src = sP + stage * C::P_BYTES + src0;
         uint8_t* dst = sB + stage * C::B_BYTES + dst0;
 #pragma unroll 4
-        for (int i = 0; i < BN / 16; ++i) {
+        for (int i = 0; i < C::B_ROWS / 16; ++i) {
           uint4 o;
           if constexpr (C::W4) {
             uint32_t h[4];
@@ -439,7 +501,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         }
         fence_proxy_async_smem();  // generic-proxy writes, read by the tensor core
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ready_bar[stage]);
+        if (lane == 0) {
+          if constexpr (C::PAIR)
+            mbar_arrive_cluster(mapa_shared(smem_u32(&ready_bar[stage]), 0));
+          else
+            mbar_arrive(&ready_bar[stage]);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
@@ -452,10 +519,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   if (warp >= 2 && warp < 2 + kEpiWarps && lane == 0) bulk_wait_group0();
   tc_fence_before();
   __syncthreads();
+  if constexpr (C::PAIR) cluster_sync_all();  // no CTA leaves while its pair may still signal it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (C::PAIR)
+      tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -463,24 +534,29 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 
 struct A16Plan {
   int bn, m_tiles, n_tiles, k_blocks, units;
+  bool pair;
   double cost;
 };
 
 // Wave-aware cost in MMA cycles: a 128 x BN x 64 fp16 block takes about
-// 2*BN cycles; a fixed charge per tile covers its epilogue tail.
-A16Plan plan_a16(int T, int N, int K, int sms, int forced_bn) {
+// 2*BN cycles; a fixed charge per tile covers its epilogue tail.  A CTA pair
+// does a 256-row unit in the time a single CTA does a 128-row one, with
+// half as many pair slots as SMs.
+A16Plan plan_a16(int T, int N, int K, int sms, int forced_bn, bool pair) {
   A16Plan best{};
   best.cost = 1e30;
   const int cands[2] = {256, 128};
+  const int slots = pair ? sms / 2 : sms;
   for (int bn : cands) {
     if (forced_bn && bn != forced_bn) continue;
     A16Plan p{};
     p.bn = bn;
-    p.m_tiles = (T + kBM - 1) / kBM;
+    p.pair = pair;
+    p.m_tiles = (T + (pair ? 2 * kBM : kBM) - 1) / (pair ? 2 * kBM : kBM);
     p.n_tiles = (N + bn - 1) / bn;
     p.k_blocks = (K + kKE - 1) / kKE;
     p.units = p.m_tiles * p.n_tiles;
-    const int waves = (p.units + sms - 1) / sms;
+    const int waves = (p.units + slots - 1) / slots;
     p.cost = waves * (p.k_blocks * 2.0 * bn + 600.0);
     if (p.cost < best.cost) best = p;
   }
@@ -500,8 +576,42 @@ cudaError_t launch_a16(const CUtensorMap& mx, const CUtensorMap& mw, const CUten
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  if constexpr (C::PAIR) {
+    // no more pairs than can be resident at once (a second, serial wave of a
+    // persistent grid would only add a tail)
+    static int max_pairs[64] = {};
+    if (dev >= 0 && dev < 64 && max_pairs[dev] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(C::NUM_THREADS);
+      cfg.dynamicSmemBytes = C::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_a16_kernel<C>, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = 1 << 20;  // unknown: keep the requested grid
+      }
+      max_pairs[dev] = n;
+    }
+    if (dev >= 0 && dev < 64) grid = std::min(grid, 2 * max_pairs[dev]);
+    return launch_pdl_cluster(gemm_a16_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
+                              static_cast<size_t>(C::SMEM_BYTES), st, 2u, mx, mw, my, p);
+  }
   return launch_pdl(gemm_a16_kernel<C>, dim3(grid), dim3(C::NUM_THREADS), C::SMEM_BYTES, st, mx,
                     mw, my, p);
+}
+
+template <bool W4, bool PAIR>
+cudaError_t dispatch_a16(int bn, const CUtensorMap& mx, const CUtensorMap& mw,
+                         const CUtensorMap& my, const A16Params& p, int grid, cudaStream_t st) {
+  return bn == 128 ? launch_a16<A16Cfg<128, W4, PAIR>>(mx, mw, my, p, grid, st)
+                   : launch_a16<A16Cfg<256, W4, PAIR>>(mx, mw, my, p, grid, st);
 }
 
 zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_grp, int g,
@@ -529,7 +639,12 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   const int fbn = option(ZQ_OPT_GEMM_BN);
   if (fbn && fbn != 128 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
   const int sms = num_sms();
-  const A16Plan plan = plan_a16(T, N, K, sms, fbn);
+  // CTA pairs halve the widening and the weight-tile traffic per SM, but the
+  // cross-CTA handshake per stage costs more than that saves (measured on
+  // B200: GPT-NeoX QKV at T = 4096 1.67 ms with pairs, 1.39 ms without), so
+  // they run only when forced (ZQ_OPT_CTA_PAIR = 2)
+  const bool pair = option(ZQ_OPT_CTA_PAIR) == 2;
+  const A16Plan plan = plan_a16(T, N, K, sms, fbn, pair);
 
   int* status = device_status_ptr();
   if (!status) return ZQ_ERR_CUDA;
@@ -556,7 +671,7 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   if (!encode_tma_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, T, static_cast<uint64_t>(K) * 2,
                      kKE, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, w_inner, N, w_inner, code_row,
-                     plan.bn, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                     plan.pair ? plan.bn / 2 : plan.bn, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !encode_tma_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
                      32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return ZQ_ERR_CUDA;
@@ -564,13 +679,17 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   int grid = std::min(plan.units, sms);
   const int cap = option(ZQ_OPT_MAX_CTAS);
   if (cap > 0) grid = std::min(grid, cap);
+  if (plan.pair) {  // an even number of CTAs, one unit per pair at a time
+    grid = 2 * std::min(plan.units, sms / 2);
+    if (cap > 0) grid = std::min(grid, std::max(2, cap & ~1));
+  }
   cudaError_t e;
-  if (w4)
-    e = plan.bn == 128 ? launch_a16<A16Cfg<128, true>>(mx, mw, my, p, grid, st)
-                       : launch_a16<A16Cfg<256, true>>(mx, mw, my, p, grid, st);
+  if (plan.pair)
+    e = w4 ? dispatch_a16<true, true>(plan.bn, mx, mw, my, p, grid, st)
+           : dispatch_a16<false, true>(plan.bn, mx, mw, my, p, grid, st);
   else
-    e = plan.bn == 128 ? launch_a16<A16Cfg<128, false>>(mx, mw, my, p, grid, st)
-                       : launch_a16<A16Cfg<256, false>>(mx, mw, my, p, grid, st);
+    e = w4 ? dispatch_a16<true, false>(plan.bn, mx, mw, my, p, grid, st)
+           : dispatch_a16<false, false>(plan.bn, mx, mw, my, p, grid, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 

@@ -498,6 +498,21 @@ def test_gemm_a16_small_t_on_tensor_cores(zq):
     _check_a16(zq, 1, 520, 256, 8, 4, seed=42, path=1)
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("T,N,K", [(16, 256, 64), (513, 1000, 256), (1024, 768, 1024), (700, 2304, 448)])
+def test_gemm_a16_cta_pairs(zq, bits, bn, T, N, K):
+    """256-row units shared by a CTA pair (cta_group::2): each CTA widens
+    half of the weight tile and keeps its 128 rows of the accumulators."""
+    _check_a16(zq, T, N, K, 8, bits, seed=bn + T + 3, bn=bn, pair=2)
+
+
+def test_gemm_a16_pairs_persistent(zq):
+    """Two pairs walk many units (both weight widths, with and without bias)."""
+    _check_a16(zq, 1500, 1536, 640, 12, 8, seed=8, bias=False, pair=2, max_ctas=4)
+    _check_a16(zq, 1500, 1536, 640, 12, 4, seed=9, pair=2, max_ctas=4)
+
+
 def test_gemm_a16_persistent_loop_and_no_bias(zq):
     """Three CTAs walk 36 tiles (two TMEM buffers and every pipeline slot
     reused many times); no bias."""

@@ -14,7 +14,10 @@
 // output, in the epilogue.
 //
 // One persistent CTA per SM walks 128 x BN output tiles (token rows on the
-// MMA M side).  Warp roles:
+// MMA M side); with ZQ_OPT_CTA_PAIR = 2 a CTA pair (cta_group::2) walks
+// 256 x BN units instead, each CTA widening half of the weight tile (built
+// and tested, but measured slower, so never chosen automatically).  Warp
+// roles:
 //   warp 0       TMA producer: per 64-element K slice, the fp16 activation
 //                tile (128 rows, 128-byte swizzle, the MMA's K-major layout)
 //                and the codes of BN weight rows (plain rows);

@@ -1,6 +1,6 @@
 """Benchmark of the fused quantized linear layer (ZeroQuant hot path) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--layer bert_base] [--tokens T]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--layer neox20b] [--tokens 4096]
     python bench.py --impl reference ...      # the CPU oracle on the host cores
 
 One step = one pass of the hot path of a transformer layer over one batch of
@@ -10,7 +10,13 @@ only where no LayerNorm precedes the GEMM) followed by the W8A8 / W4A8 GEMM
 with its fused dequant epilogue.  Weights are quantized once before timing
 (offline, as in the paper) and that time is reported separately.
 
-Prints ONE JSON line (rank 0).  `value` is int8 TOPS of the whole step
+The headline workload is the GPT-NeoX-20B layer with INT4 FFN weights and
+INT8 attention weights (g = 192) at 4096 tokens: the largest layer
+configuration, tensor-bound.  The same JSON line carries the weight-streaming
+(decode) steps of GPT-NeoX-20B at 1 and 16 tokens and GPT-J-6B at 8 and 64
+tokens, each with its weight GB/s and an HBM roofline, and the BERT-base step.
+
+Prints ONE JSON line (rank 0).  `value` is int8 TOPS of the headline step
 (2*T*N*K summed over the four GEMMs / step time) with inputs resident in HBM;
 `e2e` is the same through the C ABI with the step's fp16 inputs copied from
 pinned host memory and its fp16 outputs copied back inside the timed region.
@@ -21,6 +27,7 @@ of the flush itself (their write-back would otherwise land inside it).
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
 import json
 import os
 import statistics
@@ -32,13 +39,19 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from int4_quantized_transformer_b200 import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 INT8_PER_BF16 = 2.0  # nominal dense int8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+
+HEADLINE = ("neox20b", 4096)
+DECODE_CASES = (("neox20b", 1), ("neox20b", 16), ("gptj6b", 8), ("gptj6b", 64))
+EXTRA_PREFILL = (("bert_base", 4096),)
+
+METRIC = ("int8 TOPS of the fused quantized linear layers (LN+quant and W8A8/W4A8 GEMM with "
+          "dequant epilogue) per layer step")
 
 
 def load_peaks():
@@ -51,34 +64,25 @@ def load_peaks():
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture of the dominant GEMM with a cold L2, keyed by
-# (layer, gemm name, T); valid only for the GEMM source it was taken with
-# (sha256 prefix of csrc/gemm_i8.cu, recorded in profiles/).
-NCU_TRAFFIC = {
-    # profiles/gemm_i8_dram_traffic.md, bert_base ffn1 row (the fp16 output
-    # is still in L2 when the kernel ends, so DRAM writes read 0)
-    ("ffn1", 768, 3072, 4096): {"bytes": 5572608 + 6912, "source": "df86abc2f23b"},
-}
+# one ncu capture of a GEMM with a cold L2, keyed by (layer, gemm, T); valid
+# only for the GEMM source it was taken with (sha256 prefix of the .cu file
+# named in "file").
+NCU_TRAFFIC: dict = {}
 
 
-def _gemm_source_hash():
+def _source_hash(name: str) -> str:
     import hashlib
 
-    p = os.path.join(ROOT, "int4_quantized_transformer_b200", "csrc", "gemm_i8.cu")
+    p = os.path.join(ROOT, "int4_quantized_transformer_b200", "csrc", name)
     with open(p, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:12]
 
 
-def traffic_for(spec, T):
-    entry = NCU_TRAFFIC.get((spec.name, spec.K, spec.N, T))
-    if entry is None or entry["source"] != _gemm_source_hash():
+def traffic_for(layer, spec, T):
+    entry = NCU_TRAFFIC.get((layer, spec.name, T))
+    if entry is None or entry["source"] != _source_hash(entry["file"]):
         return None
     return entry["bytes"]
-
-
-def layer_workload(layer: str, T: int):
-    L = synth.LAYERS[layer]
-    return [synth.gemm_inputs(layer, i, T) for i in range(len(L.gemms))]
 
 
 def gemm_ops(specs, T):
@@ -87,6 +91,40 @@ def gemm_ops(specs, T):
 
 def weight_bytes(specs):
     return sum(s.N * s.K * s.bits // 8 for s in specs)
+
+
+def gemm_bytes(spec, T):
+    """Algorithmic bytes of one quantized GEMM: weights (packed for INT4),
+    int8 activations, fp16 output, fp32 scales, fp16 bias."""
+    return (spec.N * spec.K * spec.bits // 8 + T * spec.K + 2 * T * spec.N
+            + 4 * (T + spec.g) + 2 * spec.N)
+
+
+def ln_bytes(spec, T):
+    """Algorithmic bytes of one LN+quant (or quant-only) launch: fp16 rows in,
+    int8 rows and one fp32 scale per row out, gamma/beta once."""
+    return 3 * T * spec.K + 4 * T + (4 * spec.K if spec.ln else 0)
+
+
+def workload_name(layer, T, specs):
+    return (f"{layer} layer, T={T} tokens, 4 quantized linears "
+            + ", ".join(f"{s.name} {s.K}->{s.N} W{s.bits}A8 g={s.g}" for s in specs))
+
+
+def default_tokens(args):
+    """--tokens, else the layer's largest (prefill) token count."""
+    return args.tokens or max(synth.LAYERS[args.layer].tokens)
+
+
+def bench_config(layer, T, world):
+    specs = synth.LAYERS[layer].gemms
+    return {
+        "workload": workload_name(layer, T, specs),
+        "layer": layer,
+        "tokens": T,
+        "l2": "flushed before every timed step (512 MB write, then 256 MB read)",
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+    }
 
 
 # ------------------------------------------------------------------ clocks
@@ -152,30 +190,49 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ GPU arm
 
-class LayerStep:
-    """Device-resident operands and the kernel sequence of one step."""
+class LayerWeights:
+    """One layer's weights on the device: fp16 (for the cuBLAS reference
+    only), quantized codes and group scales, bias and LayerNorm parameters.
+    The synthetic weights depend on the layer and GEMM, not on T, so every
+    token count of a layer shares them."""
 
-    def __init__(self, zq, inputs, device):
-        self.zq = zq
+    def __init__(self, zq, layer, device, keep_fp16=True):
+        self.layer = layer
         self.items = []
-        for gi in inputs:
-            s = gi.spec
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for i, s in enumerate(synth.LAYERS[layer].gemms):
+            gi = synth.gemm_inputs(layer, i, 1)
             W = gi.W.to(device)
             Wq, sg = zq.quantize_weights_groupwise(W, s.g, s.bits)
-            it = {
-                "W16": W,  # the fp16 weights, for the fp16 cuBLAS comparison only
-                "spec": s,
-                "X": gi.X.to(device),
+            self.items.append({
+                "spec": s, "W16": W if keep_fp16 else None, "Wq": Wq, "s_grp": sg,
+                "b": gi.b.to(device),
                 "gamma": None if gi.gamma is None else gi.gamma.to(device),
                 "beta": None if gi.beta is None else gi.beta.to(device),
-                "Wq": Wq, "s_grp": sg, "b": gi.b.to(device),
-                "Xq": torch.empty((gi.T, s.K), dtype=torch.int8, device=device),
-                "s_tok": torch.empty(gi.T, dtype=torch.float32, device=device),
-                "Y": torch.empty((gi.T, s.N), dtype=torch.float16, device=device),
-                "T": gi.T,
-            }
-            self.items.append(it)
-        self.launches_per_step = 2 * len(self.items)
+            })
+            del W
+        torch.cuda.synchronize()
+        self.wquant_s = time.perf_counter() - t0
+
+
+class LayerStep:
+    """Device-resident operands of one layer at T tokens and the kernel
+    sequence of one step."""
+
+    def __init__(self, zq, weights: LayerWeights, T, device, inputs=None):
+        self.zq = zq
+        self.layer = weights.layer
+        self.T = T
+        self.items = []
+        for i, w in enumerate(weights.items):
+            s = w["spec"]
+            X = inputs[i].X if inputs is not None else synth.gemm_activations(self.layer, i, T)
+            self.items.append(dict(w, X=X.to(device),
+                                   Xq=torch.empty((T, s.K), dtype=torch.int8, device=device),
+                                   s_tok=torch.empty(T, dtype=torch.float32, device=device),
+                                   Y=torch.empty((T, s.N), dtype=torch.float16, device=device)))
+        self.specs = [it["spec"] for it in self.items]
 
     def run_ln(self, it, stream=None):
         self.zq.ln_quant(it["X"], it["gamma"], it["beta"], 1e-5, Xq=it["Xq"], s_tok=it["s_tok"],
@@ -248,113 +305,259 @@ def time_steps(fn, steps, flush_buf, stream):
     return total, per
 
 
+class KernelTimer:
+    """Device time of one launch sequence: a CUDA graph of R x [L2 flush,
+    body] minus a graph of R x [L2 flush], divided by R, timed with CUDA
+    events on the launching stream.  (Events between the launches of an
+    eager step would add each kernel's launch latency, which the step's
+    graph with programmatic dependent launch hides.)"""
+
+    def __init__(self, flush_buf, stream, reps):
+        self.flush_buf = flush_buf
+        self.stream = stream
+        self.reps = reps
+        self.base_ms = self._time(self._graph(None))
+
+    def _graph(self, fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(self.reps):
+                flush_l2(self.flush_buf)
+                if fn is not None:
+                    fn()
+        return g
+
+    def _time(self, g):
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        g.replay()
+        e1.record(self.stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+
+    def ms(self, fn):
+        g = self._graph(fn)
+        t = self._time(g)
+        del g
+        return max(t - self.base_ms, 1e-6) / self.reps
+
+
+def record_step(step, warmup):
+    """Warm the step up, then record it once as a CUDA graph (the paper's
+    remedy for launch overhead on small models).  Returns (graph or None,
+    error, kernel launches of one step)."""
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    n0 = step.zq.launch_count()
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step.run()
+        launches = step.zq.launch_count() - n0
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        return graph, None, launches
+    except Exception as exc:  # capture refused: report it and time eager launches
+        torch.cuda.synchronize()
+        n0 = step.zq.launch_count()
+        step.run()
+        torch.cuda.synchronize()
+        return None, f"{type(exc).__name__}: {exc}", step.zq.launch_count() - n0
+
+
+def kernel_times(step, timer):
+    kern = {}
+    for it in step.items:
+        s = it["spec"]
+        kern[(s.name, "ln")] = timer.ms(lambda it=it: step.run_ln(it))
+        kern[(s.name, "gemm")] = timer.ms(lambda it=it: step.run_gemm(it))
+    return kern
+
+
+def gemm_kernel_name(spec, T):
+    if spec.bits == 4:
+        return "gemm_i8_kernel / gemv_i8_kernel (W4A8: INT4 widened to int8 before the MMA)"
+    return "gemm_i8_kernel / gemv_i8_kernel (W8A8, tcgen05 kind::i8 or dp4a)"
+
+
+def roofline_entry(layer, spec, T, ms, peaks, peak_src, peak_tops, int8_cublas):
+    """Roofline of one GEMM launch: tensor-bound when its arithmetic intensity
+    is above the ridge point (peak ops / HBM bandwidth), else HBM-bound."""
+    ops = 2.0 * T * spec.N * spec.K
+    nbytes = gemm_bytes(spec, T)
+    hbm = float(peaks["hbm_gbs"])
+    ridge = peak_tops * 1e12 / (hbm * 1e9)
+    tensor = ops / nbytes > ridge
+    base = {"kernel": f"{gemm_kernel_name(spec, T)}, {layer} {spec.name} {spec.K}->{spec.N} "
+                      f"W{spec.bits}A8 T={T}",
+            "time_us": round(ms * 1e3, 2),
+            "traffic": traffic_for(layer, spec, T),
+            "algorithmic_bytes": nbytes, "ops": ops}
+    if tensor:
+        achieved = ops / (ms * 1e-3) / 1e12
+        r = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1),
+             "unit": "TOPS", "frac": round(achieved / peak_tops, 4),
+             "peak_source": f"{peak_src}: 2 x bf16 dense "
+                            f"{'burst' if peak_src == 'measured' else 'fallback'} "
+                            f"({peaks['bf16_tflops']} TFLOP/s), nominal int8/bf16 ratio 2"}
+        if int8_cublas:
+            r["frac_of_cublas_int8"] = round(achieved / int8_cublas, 4)
+        r["hbm_gbs_achieved"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+    else:
+        achieved = nbytes / (ms * 1e-3) / 1e9
+        r = {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(hbm, 1), "unit": "GB/s",
+             "frac": round(achieved / hbm, 4),
+             "peak_source": f"{peak_src}: copy bandwidth (hbm_gbs)",
+             "weight_gbs": round(spec.N * spec.K * spec.bits / 8 / (ms * 1e-3) / 1e9, 1),
+             "tops": round(ops / (ms * 1e-3) / 1e12, 2)}
+    r.update(base)
+    return r
+
+
+def measure_int8_peak(device, stream):
+    """cuBLAS's dense INT8 GEMM (torch._int_mm) at 8192^3, best of 10 with
+    CUDA events: a measured INT8 tensor rate on this GPU, reported next to
+    the 2 x bf16 denominator.  Returns TOPS or None."""
+    try:
+        n = 8192
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device)
+        bt = b.t()
+        for _ in range(3):
+            torch._int_mm(a, bt)
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            torch._int_mm(a, bt)
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            best = ms if best is None else min(best, ms)
+        del a, b, bt
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+
+
+def step_summary(step, kern, ms_steps, launches):
+    ops = gemm_ops(step.specs, step.T)
+    ms = sum(ms_steps) / len(ms_steps)
+    return {
+        "workload": workload_name(step.layer, step.T, step.specs),
+        "ms_per_step": round(ms, 5),
+        "ms_per_step_median": round(statistics.median(ms_steps), 5),
+        "ms_per_step_best": round(min(ms_steps), 5),
+        "tops": round(ops / (ms * 1e-3) / 1e12, 2),
+        "weight_gbs": round(weight_bytes(step.specs) / (ms * 1e-3) / 1e9, 1),
+        "gpu_launches_per_step": launches,
+        "kernels_us": {f"{n}.{k}": round(v * 1e3, 2) for (n, k), v in kern.items()},
+        "ln_quant_gbs": round(sum(ln_bytes(s, step.T) for s in step.specs)
+                              / (sum(v for (n, k), v in kern.items() if k == "ln") * 1e-3) / 1e9, 1),
+    }
+
+
+def dominant_gemm(step, kern):
+    it = max(step.items, key=lambda it: kern[(it["spec"].name, "gemm")])
+    return it["spec"], kern[(it["spec"].name, "gemm")]
+
+
+def fp16_reference(step, timer, with_int8=False):
+    """Library references, measured after this library's kernels: the same
+    GEMM shapes in fp16 through cuBLAS (torch.addmm: X W^T + b), per GEMM and
+    as a graph of the fp16 layer (torch layer_norm before the GEMMs that have
+    a LayerNorm), and cuBLAS's INT8 GEMM (torch._int_mm, int32 out, no
+    scales) on the dominant shape.  Context, not part of the path."""
+    out = {}
+    try:
+        fns = [lambda it=it: torch.addmm(it["b"], it["X"], it["W16"].t()) for it in step.items]
+        for fn in fns:
+            fn()  # cuBLAS sets up its handle and workspace outside any capture
+        torch.cuda.synchronize()
+        per = {it["spec"].name: timer.ms(fn) for it, fn in zip(step.items, fns)}
+
+        def fp16_layer():
+            for it in step.items:
+                x = it["X"]
+                if it["gamma"] is not None:
+                    x = torch.nn.functional.layer_norm(x, (x.shape[1],), it["gamma"], it["beta"],
+                                                       1e-5)
+                torch.addmm(it["b"], x, it["W16"].t())
+
+        fp16_layer()
+        torch.cuda.synchronize()
+        out = {"gemm_us": {n: round(v * 1e3, 2) for n, v in per.items()},
+               "step_us": round(timer.ms(fp16_layer) * 1e3, 2)}
+        if with_int8 and step.T > 16:
+            it = max(step.items, key=lambda it: it["spec"].N * it["spec"].K)
+            s = it["spec"]
+            x8 = torch.randint(-127, 128, (step.T, s.K), dtype=torch.int8, device=it["X"].device)
+            w8 = torch.randint(-127, 128, (s.N, s.K), dtype=torch.int8, device=it["X"].device)
+            torch._int_mm(x8, w8.t())
+            torch.cuda.synchronize()
+            out["cublas_int8_us"] = {s.name: round(timer.ms(lambda: torch._int_mm(x8, w8.t())) * 1e3,
+                                                   2)}
+    except Exception as exc:
+        torch.cuda.synchronize()
+        out = {"error": f"{type(exc).__name__}: {exc}"}
+    return out
+
+
+def measure_step(zq, weights, T, args, timer, flush_buf, stream, dist_on, inputs=None):
+    """Build one layer step at T tokens, record it as a graph, time K steps
+    (L2 flushed before each) and every kernel on its own."""
+    step = LayerStep(zq, weights, T, torch.device("cuda", torch.cuda.current_device()), inputs)
+    graph, graph_error, launches = record_step(step, args.warmup)
+    run_step = graph.replay if graph is not None else step.run
+    barrier(dist_on)
+    total_ms, per_step = time_steps(run_step, args.steps, flush_buf, stream)
+    barrier(dist_on)
+    total_ms = max_over_ranks(total_ms, dist_on)
+    kern = kernel_times(step, timer)
+    return step, graph, graph_error, launches, total_ms / args.steps, per_step, kern
+
+
 def gpu_arm(args, dist_on, rank, world):
     from int4_quantized_transformer_b200 import zq
 
     device = torch.device("cuda", torch.cuda.current_device())
     peaks, peak_src = load_peaks()
-    layer = args.layer
-    T = args.tokens or synth.LAYERS[layer].tokens[0]
-    inputs = layer_workload(layer, T)
-    specs = [gi.spec for gi in inputs]
-    ops = gemm_ops(specs, T)
-    wbytes = weight_bytes(specs)
+    peak_tops = INT8_PER_BF16 * float(peaks["bf16_tflops"])
+    layer, T = args.layer, default_tokens(args)
     stream = torch.cuda.current_stream()
-
-    # offline weight quantization (timed once, reported separately)
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    step = LayerStep(zq, inputs, device)
-    torch.cuda.synchronize()
-    wquant_s = time.perf_counter() - t0
     flush_buf = make_flush_buffers(device)
+    timer = KernelTimer(flush_buf, stream, max(3, min(args.steps, 20)))
 
-    for _ in range(args.warmup):
-        step.run()
+    # ---- the headline step: inputs resident in HBM, K steps timed
+    cpu_inputs = [synth.gemm_inputs(layer, i, T) for i in range(len(synth.LAYERS[layer].gemms))]
+    weights = LayerWeights(zq, layer, device)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step, graph, graph_error, launches, ms_per_step, per_step, kern = measure_step(
+            zq, weights, T, args, timer, flush_buf, stream, dist_on, inputs=cpu_inputs)
     rc, detail = zq.device_status()
     if rc != zq.ZQ_OK:
-        raise RuntimeError(f"device status {rc} ({detail}) after warm-up")
-
-    # The step's kernel sequence is recorded once as a CUDA graph and replayed
-    # (the paper's remedy for launch overhead on small models, Appendix D).
-    graph = None
-    graph_error = None
-    if not args.eager:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                step.run()
-            for _ in range(args.warmup):
-                graph.replay()
-        except Exception as exc:  # capture refused: report it and time eager launches
-            graph, graph_error = None, f"{type(exc).__name__}: {exc}"
-            torch.cuda.synchronize()
+        raise RuntimeError(f"device status {rc} ({detail}) after timing")
     run_step = graph.replay if graph is not None else step.run
-
-    # ---- timed region: K steps, inputs resident in HBM
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        barrier(dist_on)
-        total_ms, per_step = time_steps(run_step, args.steps, flush_buf, stream)
-        barrier(dist_on)
-    total_ms = max_over_ranks(total_ms, dist_on)
-    ms_per_step = total_ms / args.steps
+    specs = step.specs
+    ops = gemm_ops(specs, T)
     eager_ms, _ = time_steps(step.run, max(3, args.steps // 2), flush_buf, stream)
     eager_ms /= max(3, args.steps // 2)
+    int8_cublas = measure_int8_peak(device, stream)
 
-    # ---- per-kernel device times for the roofline: a CUDA graph of R x
-    # [L2 flush, kernel] minus a graph of R x [L2 flush], divided by R, both
-    # timed with CUDA events on the launching stream.  (Events between the
-    # launches of an eager step would also count each kernel's launch
-    # latency, which the step's graph with programmatic dependent launch
-    # hides.)
-    reps = max(3, min(args.steps, 20))
-
-    def graph_of(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for _ in range(reps):
-                flush_l2(flush_buf)
-                if fn is not None:
-                    fn()
-        return g
-
-    def time_graph(g):
-        g.replay()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1)
-
-    kern = {}
-    try:
-        base_ms = time_graph(graph_of(None))
-        for it in step.items:
-            s = it["spec"]
-            for kind in ("ln", "gemm"):
-                fn = (lambda it=it: step.run_ln(it)) if kind == "ln" else (lambda it=it: step.run_gemm(it))
-                kern[(s.name, kind)] = max(time_graph(graph_of(fn)) - base_ms, 1e-6) / reps
-        kern_method = f"CUDA graph of {reps} x [L2 flush, kernel] minus {reps} x [L2 flush]"
-    except Exception as exc:  # graphs refused: eager launches after a flush
-        torch.cuda.synchronize()
-        for it in step.items:
-            s = it["spec"]
-            for kind in ("ln", "gemm"):
-                fn = (lambda it=it: step.run_ln(it)) if kind == "ln" else (lambda it=it: step.run_gemm(it))
-                tot, _ = time_steps(fn, reps, flush_buf, stream)
-                kern[(s.name, kind)] = tot / reps
-        kern_method = f"eager launches after an L2 flush ({type(exc).__name__})"
+    dom_spec, dom_ms = dominant_gemm(step, kern)
     gemm_ms = sum(v for (n, k), v in kern.items() if k == "gemm")
-    ln_ms = sum(v for (n, k), v in kern.items() if k == "ln")
-    peak_tops = INT8_PER_BF16 * float(peaks["bf16_tflops"])
-    # the dominant kernel: the GEMM launch with the largest device time
-    dom = max((it for it in step.items), key=lambda it: kern[(it["spec"].name, "gemm")])
-    dom_spec = dom["spec"]
-    dom_ms = kern[(dom_spec.name, "gemm")]
-    dom_ops = 2.0 * T * dom_spec.N * dom_spec.K
-    achieved_tops = dom_ops / (dom_ms * 1e-3) / 1e12
-    all_gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    roof = roofline_entry(layer, dom_spec, T, dom_ms, peaks, peak_src, peak_tops, int8_cublas)
+    roof["all_gemms_tops"] = round(ops / (gemm_ms * 1e-3) / 1e12, 1)
+    roof["kernel_time_method"] = (f"CUDA graph of {timer.reps} x [L2 flush, kernel] minus "
+                                  f"{timer.reps} x [L2 flush]")
+    roof["int8_cublas_8192_tops"] = None if int8_cublas is None else round(int8_cublas, 1)
+    per_gemm = {s.name: roofline_entry(layer, s, T, kern[(s.name, "gemm")], peaks, peak_src,
+                                       peak_tops, int8_cublas) for s in specs}
 
     # ---- end to end through the C ABI: pinned host inputs in, outputs out
     h_in = [it["X"].cpu().pin_memory() for it in step.items]
@@ -363,10 +566,10 @@ def gpu_arm(args, dist_on, rank, world):
     d2h = sum(y.numel() * 2 for y in h_out)
 
     def e2e_step():
-        for it, hx, hy in zip(step.items, h_in, h_out):
+        for it, hx in zip(step.items, h_in):
             it["X"].copy_(hx, non_blocking=True)
         run_step()
-        for it, hx, hy in zip(step.items, h_in, h_out):
+        for it, hy in zip(step.items, h_out):
             hy.copy_(it["Y"], non_blocking=True)
 
     for _ in range(2):
@@ -375,133 +578,127 @@ def gpu_arm(args, dist_on, rank, world):
     e2e_ms, _ = time_steps(e2e_step, args.steps, flush_buf, stream)
     barrier(dist_on)
     e2e_ms = max_over_ranks(e2e_ms, dist_on) / args.steps
+    del h_in, h_out
+
+    fp16 = fp16_reference(step, timer, with_int8=True)
+    if "gemm_us" in fp16:
+        fp16["gemm_speedup"] = round(sum(fp16["gemm_us"].values()) / (gemm_ms * 1e3), 3)
+        fp16["step_speedup"] = round(fp16["step_us"] / (ms_per_step * 1e3), 3)
+    wquant_ms = weights.wquant_s * 1e3
+    summary = step_summary(step, kern, per_step, launches)
+    del graph, step
+
+    # ---- weight-streaming (decode) steps and the smaller prefill layer:
+    # every GEMM gets its roofline (HBM at these token counts)
+    decode = {}
+    extra = {}
+    if not args.no_decode:
+        for dl, dT in DECODE_CASES:
+            if weights.layer != dl:
+                del weights
+                torch.cuda.empty_cache()
+                weights = LayerWeights(zq, dl, device)
+            st, g, _, la, ms, per, kn = measure_step(zq, weights, dT, args, timer, flush_buf,
+                                                     stream, dist_on)
+            d = step_summary(st, kn, per, la)
+            ds, dms = dominant_gemm(st, kn)
+            d["roofline"] = roofline_entry(dl, ds, dT, dms, peaks, peak_src, peak_tops, int8_cublas)
+            d["gemms"] = {s.name: roofline_entry(dl, s, dT, kn[(s.name, "gemm")], peaks, peak_src,
+                                                 peak_tops, int8_cublas) for s in st.specs}
+            d["fp16_cublas"] = fp16_reference(st, timer)
+            decode[f"{dl}_T{dT}"] = d
+            del st, g
+        for el, eT in EXTRA_PREFILL:
+            del weights
+            torch.cuda.empty_cache()
+            weights = LayerWeights(zq, el, device)
+            st, g, _, la, ms, per, kn = measure_step(zq, weights, eT, args, timer, flush_buf, stream,
+                                                     dist_on)
+            d = step_summary(st, kn, per, la)
+            ds, dms = dominant_gemm(st, kn)
+            d["roofline"] = roofline_entry(el, ds, eT, dms, peaks, peak_src, peak_tops, int8_cublas)
+            d["fp16_cublas"] = fp16_reference(st, timer)
+            extra[f"{el}_T{eT}"] = d
+            del st, g
     rc, detail = zq.device_status()
     if rc != zq.ZQ_OK:
-        raise RuntimeError(f"device status {rc} ({detail}) after timing")
+        raise RuntimeError(f"device status {rc} ({detail}) after the decode steps")
 
-    # ---- library references, measured last so that nothing above runs after
-    # cuBLAS work or its graph captures: the same shapes in fp16 through cuBLAS
-    # (torch.addmm: X W^T + b), per GEMM and as a graph of the four GEMMs, and
-    # cuBLAS's own INT8 GEMM (torch._int_mm, int32 out, no scales) on the
-    # dominant shape, timed like the kernels above
-    ref16, ref16_step_ms, ref_i8, ref16_error = {}, None, None, None
-    try:
-        fns16 = [lambda it=it: torch.addmm(it["b"], it["X"], it["W16"].t()) for it in step.items]
-        for fn16 in fns16:
-            fn16()  # cuBLAS sets up its handle and workspace outside any capture
-        torch.cuda.synchronize()
-        for it, fn16 in zip(step.items, fns16):
-            ref16[it["spec"].name] = max(time_graph(graph_of(fn16)) - base_ms, 1e-6) / reps
-        # the fp16 layer: LayerNorm before the GEMMs that have one, then the GEMM
-        def fp16_layer():
-            for it in step.items:
-                x = it["X"]
-                if it["gamma"] is not None:
-                    x = torch.nn.functional.layer_norm(x, (x.shape[1],), it["gamma"], it["beta"], 1e-5)
-                torch.addmm(it["b"], x, it["W16"].t())
-
-        fp16_layer()
-        torch.cuda.synchronize()
-        ref16_step_ms = max(time_graph(graph_of(fp16_layer)) - base_ms, 1e-6) / reps
-        if T > 16:
-            x8 = torch.randint(-127, 128, (T, dom_spec.K), dtype=torch.int8, device=device)
-            w8 = torch.randint(-127, 128, (dom_spec.N, dom_spec.K), dtype=torch.int8, device=device)
-            torch._int_mm(x8, w8.t())
-            torch.cuda.synchronize()
-            ref_i8 = max(time_graph(graph_of(lambda: torch._int_mm(x8, w8.t()))) - base_ms,
-                         1e-6) / reps
-    except Exception as exc:
-        torch.cuda.synchronize()
-        ref16_error = f"{type(exc).__name__}: {exc}"
-
+    cfg = bench_config(layer, T, world)
+    cfg["launch"] = "cuda graph replay of the step" if graph_error is None else "eager launches"
     res = {
-        "metric": "int8 TOPS of the fused quantized linear layers (LN+quant and W8A8/W4A8 GEMM "
-                  "with dequant epilogue) per layer step",
+        "metric": METRIC,
         "value": round(whole_job_tops(ops, world, ms_per_step), 2),
         "unit": "TOPS",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5),
-        "ms_per_step_median": round(statistics.median(per_step), 5),
-        "ms_per_step_best": round(min(per_step), 5),
+        "ms_per_step_median": summary["ms_per_step_median"],
+        "ms_per_step_best": summary["ms_per_step_best"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "int8",
         "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,sigma) weights)",
-        "config": {
-            "workload": f"{layer} layer, T={T} tokens, 4 quantized linears "
-                        + ", ".join(f"{s.name} {s.K}->{s.N} W{s.bits}A8 g={s.g}" for s in specs),
-            "tokens": T,
-            "l2": "flushed before every timed step (512 MB write, then 256 MB read)",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "launch": "cuda graph replay of the step" if graph is not None else "eager launches",
-        },
+        "config": cfg,
         "eager_ms_per_step": round(eager_ms, 5),
         "graph_error": graph_error,
-        "weight_gbs": round(world * wbytes / (ms_per_step * 1e-3) / 1e9, 1),
-        "roofline": {
-            "bound": "tensor",
-            "kernel": f"gemm_i8_kernel (tcgen05 kind::i8), {dom_spec.name} {dom_spec.K}->{dom_spec.N} "
-                      f"T={T}",
-            "achieved": round(achieved_tops, 1),
-            "peak": round(peak_tops, 1),
-            "unit": "TOPS",
-            "frac": round(achieved_tops / peak_tops, 4),
-            "peak_source": f"{peak_src}: 2 x bf16 dense {'burst' if peak_src == 'measured' else 'fallback'} "
-                           f"({peaks['bf16_tflops']} TFLOP/s), nominal int8/bf16 ratio 2",
-            "traffic": traffic_for(dom_spec, T),
-            "all_gemms_tops": round(all_gemm_tops, 1),
-            "kernel_time_method": kern_method,
-        },
-        "kernels_us": {f"{n}.{k}": round(v * 1e3, 2) for (n, k), v in kern.items()},
-        "fp16_cublas": {"error": ref16_error} if not ref16 else {
-            "what": "torch.addmm(bias, X, W^T) in fp16 (cuBLAS) on each GEMM shape of the step, "
-                    "timed as the kernels above; step = a graph of the fp16 layer (torch layer_norm "
-                    "before the GEMMs that have a LayerNorm, then the four GEMMs), L2 flushed before it",
-            "gemm_us": {n: round(v * 1e3, 2) for n, v in ref16.items()},
-            "step_us": None if ref16_step_ms is None else round(ref16_step_ms * 1e3, 2),
-            "gemm_speedup": round(sum(ref16.values()) / gemm_ms, 3),
-            "step_speedup": None if ref16_step_ms is None else round(ref16_step_ms / ms_per_step, 3),
-            "dominant_fp16_tflops": round(dom_ops / (ref16[dom_spec.name] * 1e-3) / 1e12, 1),
-            "dominant_cublas_int8_us": None if ref_i8 is None else round(ref_i8 * 1e3, 2),
-        },
-        "ln_quant_gbs": round(sum(3 * it["T"] * it["spec"].K for it in step.items) / (ln_ms * 1e-3) / 1e9, 1),
-        "offline_wquant_ms": round(wquant_s * 1e3, 2),
+        "weight_gbs": round(world * weight_bytes(specs) / (ms_per_step * 1e-3) / 1e9, 1),
+        "roofline": roof,
+        "gemms": per_gemm,
+        "kernels_us": summary["kernels_us"],
+        "ln_quant_gbs": summary["ln_quant_gbs"],
+        "fp16_cublas": fp16,
+        "decode": decode,
+        "extra_prefill": extra,
+        "offline_wquant_ms": round(wquant_ms, 2),
         "e2e": {"value": round(whole_job_tops(ops, world, e2e_ms), 2), "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step.launches_per_step * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        res["cpu_baseline"] = cpu_baseline(layer, T, args.cpu_tokens)
+        res["cpu_baseline"] = cpu_baseline(layer, T, args.cpu_tokens, args.cpu_tokens_1,
+                                           cpu_inputs)
     return res
 
 
 # ------------------------------------------------------------------ CPU oracle arm
 
-def oracle_step(inputs, rows):
-    """The oracle's hot path on a token subset: ln_quant + exact GEMM + dequant."""
+def prepare_oracle(layer, T, inputs=None):
     import oracle
 
-    for gi in inputs:
-        s = gi.spec
-        X = gi.X.numpy()[:rows]
-        xq, st = oracle.ln_quant(X, None if gi.gamma is None else gi.gamma.numpy(),
-                                 None if gi.beta is None else gi.beta.numpy(), 1e-5)
-        wq, sg = gi.extra["wq"], gi.extra["sg"]
-        oracle.linear_q(xq, st, wq, sg, gi.b.numpy())
-
-
-def prepare_oracle(layer, T):
-    import oracle
-
-    inputs = layer_workload(layer, T)
+    inputs = inputs or [synth.gemm_inputs(layer, i, T)
+                        for i in range(len(synth.LAYERS[layer].gemms))]
+    ready = []
     for gi in inputs:
         wq, sg = oracle.quantize_weights_groupwise(gi.W.numpy(), gi.spec.g, gi.spec.bits)
-        gi.extra["wq"], gi.extra["sg"] = wq, sg
-    return inputs
+        ready.append({"spec": gi.spec, "X": gi.X.numpy(), "wq": wq, "sg": sg, "b": gi.b.numpy(),
+                      "gamma": None if gi.gamma is None else gi.gamma.numpy(),
+                      "beta": None if gi.beta is None else gi.beta.numpy()})
+    return ready
+
+
+def _oracle_rows(g, r0, r1):
+    import oracle
+
+    xq, st = oracle.ln_quant(g["X"][r0:r1], g["gamma"], g["beta"], 1e-5)
+    oracle.linear_q(xq, st, g["wq"], g["sg"], g["b"])
+
+
+def oracle_step(ready, rows, pool=None, threads=1):
+    """The oracle's hot path on the first `rows` tokens: LN+quant, exact int
+    GEMM, dequant, for every GEMM of the layer.  With a thread pool the rows
+    are split into `threads` contiguous chunks (the C oracle runs without the
+    interpreter lock, so the chunks run on separate cores)."""
+    for g in ready:
+        if pool is None:
+            _oracle_rows(g, 0, rows)
+            continue
+        cuts = [rows * i // threads for i in range(threads + 1)]
+        list(pool.map(lambda ab: _oracle_rows(g, *ab),
+                      [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]))
 
 
 def host_cpu_model() -> str:
@@ -515,47 +712,67 @@ def host_cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(layer, T, rows):
-    rows = min(rows, T)
-    inputs = prepare_oracle(layer, T)
+def _host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(layer, T, rows_all, rows_one, inputs=None):
+    """The oracle as it stands on the host cores: all cores (threads over
+    token-row chunks) and one core, each on a bounded token sample."""
+    ready = prepare_oracle(layer, T, inputs)
+    specs = [g["spec"] for g in ready]
+    threads = _host_threads()
+    rows_all = min(rows_all, T)
+    rows_one = min(rows_one, T)
+    with cf.ThreadPoolExecutor(max_workers=threads) as pool:
+        t0 = time.perf_counter()
+        oracle_step(ready, rows_all, pool, threads)
+        dt_all = time.perf_counter() - t0
     t0 = time.perf_counter()
-    oracle_step(inputs, rows)
-    dt = time.perf_counter() - t0
-    ops = gemm_ops([gi.spec for gi in inputs], rows)
-    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "host_cpu_model": host_cpu_model(),
-            "sample": f"{rows} of {T} tokens of every GEMM of the step (LN+quant, exact int GEMM, "
-                      f"dequant), single-threaded plain C, {dt:.1f} s",
-            "host_cpus": os.cpu_count()}
+    oracle_step(ready, rows_one)
+    dt_one = time.perf_counter() - t0
+    v_all = gemm_ops(specs, rows_all) / dt_all / 1e12
+    v_one = gemm_ops(specs, rows_one) / dt_one / 1e12
+    return {"value": round(v_all, 6), "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{rows_all} of {T} tokens of every GEMM of the {layer} step (LN+quant, exact "
+                      f"int GEMM, dequant), plain C on {threads} threads over token-row chunks, "
+                      f"{dt_all:.1f} s",
+            "single_core": {"value": round(v_one, 6), "unit": "TOPS", "cores": 1,
+                            "sample": f"{rows_one} of {T} tokens of every GEMM, single-threaded, "
+                                      f"{dt_one:.1f} s"},
+            "host_cpu_model": host_cpu_model(), "host_cpus": os.cpu_count()}
 
 
 def reference_arm(args, rank, world):
-    layer = args.layer
-    T = args.tokens or synth.LAYERS[layer].tokens[0]
+    layer, T = args.layer, default_tokens(args)
     rows = min(args.ref_tokens, T)
-    inputs = prepare_oracle(layer, T)
-    specs = [gi.spec for gi in inputs]
-    for _ in range(args.warmup):
-        oracle_step(inputs, rows)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_step(inputs, rows)
-    dt = (time.perf_counter() - t0) / args.steps
-    ops = gemm_ops(specs, rows)
-    val = round(ops / dt / 1e12, 6)
-    sample = (f"{rows} of {T} tokens of every GEMM of the {layer} step per timed step "
-              f"(oracle: LN+quant, exact int GEMM, dequant), single-threaded plain C")
+    ready = prepare_oracle(layer, T)
+    specs = [g["spec"] for g in ready]
+    threads = _host_threads()
+    with cf.ThreadPoolExecutor(max_workers=threads) as pool:
+        for _ in range(args.warmup):
+            oracle_step(ready, rows, pool, threads)
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle_step(ready, rows, pool, threads)
+        dt = (time.perf_counter() - t0) / args.steps
+    val = round(gemm_ops(specs, rows) / dt / 1e12, 6)
+    sample = (f"{rows} of {T} tokens of every GEMM of the {layer} step per timed step (oracle: "
+              f"LN+quant, exact int GEMM, dequant), plain C on {threads} threads over token-row "
+              f"chunks")
     return {
         "impl": "reference",
-        "metric": "int8 TOPS of the fused quantized linear layers (LN+quant and W8A8/W4A8 GEMM "
-                  "with dequant epilogue) per layer step",
+        "metric": METRIC,
         "value": val, "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": f"{layer} layer, T={T} tokens (oracle timed on a {rows}-token sample)",
-                   "tokens": T},
-        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": 1, "kind": "oracle", "sample": sample,
-                         "host_cpu_model": host_cpu_model(), "host_cpus": os.cpu_count()},
+        "config": bench_config(layer, T, world),
+        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                         "sample": sample, "host_cpu_model": host_cpu_model(),
+                         "host_cpus": os.cpu_count()},
         "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -563,15 +780,20 @@ def reference_arm(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="zq", choices=["zq", "reference"])
-    ap.add_argument("--layer", default="bert_base", choices=sorted(synth.LAYERS))
+    ap.add_argument("--layer", default=HEADLINE[0], choices=sorted(synth.LAYERS))
     ap.add_argument("--tokens", type=int, default=0)
-    ap.add_argument("--cpu-tokens", type=int, default=2048)
-    ap.add_argument("--ref-tokens", type=int, default=64)
+    ap.add_argument("--cpu-tokens", type=int, default=256,
+                    help="token sample of the all-core CPU baseline")
+    ap.add_argument("--cpu-tokens-1", type=int, default=32,
+                    help="token sample of the single-core CPU baseline")
+    ap.add_argument("--ref-tokens", type=int, default=32,
+                    help="token sample per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--eager", action="store_true", help="launch kernels one by one (no CUDA graph)")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode steps and the extra prefill layer")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

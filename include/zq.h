@@ -271,6 +271,14 @@ zq_status zq_set_option(int key, int value);
 int zq_get_option(int key);
 
 /*
+ * zq_launch_count -- number of kernel launches this library has issued in
+ * this process, on every device and stream (a launch recorded into a CUDA
+ * graph counts once, when it is recorded; its replays do not go through the
+ * library).  Benchmarks use the difference over one recorded step.
+ */
+unsigned long long zq_launch_count(void);
+
+/*
  * zq_debug_wait_timeout -- launches one CTA that waits on a shared-memory
  * barrier nothing ever arrives at.  The wait is bounded: after about a
  * second it records ZQ_ERR_TIMEOUT in the status word and the kernel

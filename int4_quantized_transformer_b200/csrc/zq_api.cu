@@ -21,6 +21,7 @@ std::mutex g_mu;
 int* g_status_ptr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
 std::atomic<int> g_opts[8];
+std::atomic<unsigned long long> g_launches{0};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int current_device() {
@@ -54,6 +55,8 @@ int num_sms() {
   }
   return g_num_sms[d];
 }
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int option(int key) {
   if (key < 1 || key >= 8) return 0;
@@ -118,7 +121,7 @@ const char* zq_status_str(int s) {
   }
 }
 
-int zq_abi_version(void) { return 103; }
+int zq_abi_version(void) { return 104; }
 
 zq_status zq_set_option(int key, int value) {
   if (key < ZQ_OPT_GEMM_PATH || key > ZQ_OPT_CTA_PAIR) return ZQ_ERR_UNSUPPORTED;
@@ -131,6 +134,8 @@ zq_status zq_set_option(int key, int value) {
 }
 
 int zq_get_option(int key) { return option(key); }
+
+unsigned long long zq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 zq_status zq_device_status(zq_stream_t stream, int* detail) {
   if (detail) *detail = 0;
@@ -149,6 +154,7 @@ zq_status zq_device_status(zq_stream_t stream, int* detail) {
 zq_status zq_debug_wait_timeout(zq_stream_t stream) {
   int* st = device_status_ptr();
   if (!st) return ZQ_ERR_CUDA;
+  count_launch();
   debug_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(st);
   ZQ_CUDA_OK(cudaGetLastError());
   return ZQ_OK;

@@ -33,6 +33,8 @@ cudaError_t launch_gemv_a16(int bits, const void* X, const void* W, const float*
                             const void* bias, int T, int N, int K, void* Y, float* acc_dbg,
                             int max_ctas, cudaStream_t st);
 int option(int key);
+// Counts one kernel launch issued by the library (zq_launch_count).
+void count_launch();
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 // Returns false when the driver entry point is unavailable or encoding fails.
@@ -59,6 +61,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  count_launch();
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -81,6 +84,7 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  count_launch();
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 

@@ -134,6 +134,17 @@ class GemmInputs:
     extra: dict = field(default_factory=dict)
 
 
+def gemm_activations(layer: str, gemm_index: int, T: int) -> torch.Tensor:
+    """The seeded fp16 input rows [T, K] of one GEMM of one layer: the X of
+    gemm_inputs, without drawing the weights."""
+    L = LAYERS[layer]
+    s = L.gemms[gemm_index]
+    if layer == "tiny":
+        return activations(T, s.K, 0)
+    base = L.seed_base + 10 * gemm_index
+    return activations(T, s.K, base + 1, L.n_outliers(s.K), L.outlier_scale)
+
+
 def gemm_inputs(layer: str, gemm_index: int, T: int) -> GemmInputs:
     """Seeded inputs of one GEMM of one layer (sub-seed = base + 10*index + tensor)."""
     L = LAYERS[layer]
@@ -144,7 +155,7 @@ def gemm_inputs(layer: str, gemm_index: int, T: int) -> GemmInputs:
         W = weights(s.N, s.K, L.sigma_w, 1)
         b = bias(s.N, 2)
         return GemmInputs(s, T, X, W, b)
-    X = activations(T, s.K, base + 1, L.n_outliers(s.K), L.outlier_scale)
+    X = gemm_activations(layer, gemm_index, T)
     W = weights(s.N, s.K, L.sigma_w, base + 2)
     b = bias(s.N, base + 3)
     gamma = beta = None

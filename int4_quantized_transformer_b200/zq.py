@@ -24,7 +24,7 @@ EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
     "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant", "zq_static_quant",
-    "zq_gemm_w8a16", "zq_gemm_w4a16",
+    "zq_gemm_w8a16", "zq_gemm_w4a16", "zq_launch_count",
 )
 
 
@@ -56,6 +56,7 @@ def _load():
         "zq_static_quant": ([P, I, I, F, P, P, P], I),
         "zq_gemm_w8a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
         "zq_gemm_w4a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
+        "zq_launch_count": ([], ctypes.c_ulonglong),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -101,6 +102,11 @@ def _dev(t: torch.Tensor | None, dtype, shape, name: str):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def launch_count() -> int:
+    """Kernel launches this library has issued in this process (zq_launch_count)."""
+    return int(_lib.zq_launch_count())
 
 
 def set_option(key: int, value: int):

@@ -7,6 +7,10 @@ import subprocess
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
 
 
 def _run(extra_env, *args):
@@ -16,7 +20,7 @@ def _run(extra_env, *args):
 
 
 def test_reference_arm_prints_the_contract_line():
-    out = _run({}, "--steps", "2", "--warmup", "3", "--ref-tokens", "4")
+    out = _run({}, "--steps", "2", "--warmup", "3", "--ref-tokens", "4", "--layer", "tiny")
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -29,13 +33,16 @@ def test_reference_arm_prints_the_contract_line():
     assert d["steps"] == 2 and d["warmup"] == 3
     assert d["value"] > 0 and d["higher_is_better"] is True
     assert "workload" in d["config"]
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    # the reference line describes the same workload as the GPU arm's line
+    assert d["config"] == bench.bench_config("tiny", 16, 1)
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
 
 
 def test_reference_arm_is_silent_on_other_ranks():
-    out = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, "--steps", "1", "--ref-tokens", "2")
+    out = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, "--steps", "1", "--ref-tokens", "2",
+               "--layer", "tiny")
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip() == ""

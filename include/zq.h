@@ -19,9 +19,12 @@
  *    the fact in a per-device status word that zq_device_status() reports.
  *  - Group of output row o when N rows are split into g contiguous groups:
  *    group(o) = floor(o*g/N).
- *  - Rounding: round half to even everywhere; every floating-point step is a
- *    single IEEE round-to-nearest operation (no fused multiply-add), so the
- *    results are bit-for-bit reproducible.
+ *  - Rounding: round half to even everywhere.  Every floating-point step is
+ *    one IEEE round-to-nearest operation in a stated order: a single add,
+ *    multiply, divide or square root, except in the LayerNorm variance, whose
+ *    squared deviations are accumulated with fused multiply-adds (one
+ *    rounding each).  Results are therefore bit-for-bit reproducible and do
+ *    not depend on the launch configuration.
  */
 #ifndef ZQ_H_
 #define ZQ_H_

@@ -374,8 +374,18 @@ def test_repeated_split_k_calls_leave_workspace_clean(zq):
 # ------------------------------------------------------------ full-size configurations
 
 def _sample_rows(T, n=6):
-    rows = sorted(set([0, T - 1] + list(np.random.default_rng(T).integers(0, T, n))))
-    return np.array(rows)
+    """Token rows at every tiling edge of the plans the GEMMs choose, plus
+    random ones: the first and last row of 16- to 256-row token tiles around
+    the start, of the last 128-row tile and of both 128-row halves of the
+    last 256-row CTA-pair tile, and T - 1."""
+    edges = {0, T - 1}
+    for b in (16, 32, 64, 128, 256, 512):
+        edges |= {b - 1, b}
+    for tile in (128, 256):
+        last = (T - 1) // tile * tile
+        edges |= {last - 1, last, min(last + 127, T - 1), last + 128}
+    rnd = np.random.default_rng(T).integers(0, T, n)
+    return np.array(sorted(r for r in edges | set(int(v) for v in rnd) if 0 <= r < T))
 
 
 FULL = [(layer, gi, T) for layer in ("bert_base", "gpt350m", "gptj6b", "neox20b")
@@ -410,6 +420,20 @@ def test_full_size_sampled_rows(zq, layer, gi, T):
     acc = oracle.gemm_i32(xq, wq)
     assert_bits_equal(host(acc_d)[rows], acc)
     assert_fp16_close(host(Y_d)[rows], oracle.dequant(acc, st, sg, inp.b.numpy()))
+    if layer == "neox20b" and T == 4096 and s.bits == 4:
+        # INT4 weights at prefill size: every token of the first and the last
+        # 128-row weight tile (one output stripe each), against the oracle
+        xq_all, st_all = oracle.ln_quant(inp.X.numpy(),
+                                         None if inp.gamma is None else inp.gamma.numpy(),
+                                         None if inp.beta is None else inp.beta.numpy(), 1e-5)
+        assert_bits_equal(host(xq_d), xq_all)
+        for c0 in (0, s.N - 128):
+            cols = slice(c0, c0 + 128)
+            acc_s = oracle.gemm_i32(xq_all, wq[cols])
+            assert_bits_equal(host(acc_d)[:, cols], acc_s)
+            sg_cols = sg[oracle.group_index(s.N, s.g)[cols]]
+            ref = oracle.dequant(acc_s, st_all, sg_cols, inp.b.numpy()[cols])
+            assert_fp16_close(host(Y_d)[:, cols], ref)
 
 
 # ------------------------------------------------------------ FP16 activations (W8A16 / W4A16)
@@ -556,7 +580,7 @@ def test_gemm_a16_full_size_sampled_rows(zq, layer, gi, T, bits):
     acc_d = torch.empty((T, s.N), dtype=torch.float32, device="cuda")
     fn = zq.gemm_w4a16 if bits == 4 else zq.gemm_w8a16
     Y = fn(dev(inp.X), wdev, torch.from_numpy(sg).cuda(), dev(inp.b), acc_dbg=acc_d)
-    rows = _sample_rows(T)[:6]
+    rows = _sample_rows(T, n=2)
     Xs = inp.X.numpy()[rows]
     acc_ref, y_ref, Y_ref = oracle.gemm_a16(Xs, wq, sg, inp.b.numpy())
     _assert_a16_close(Xs, wq, sg, host(acc_d)[rows], host(Y)[rows], acc_ref, y_ref, Y_ref)

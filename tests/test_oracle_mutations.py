@@ -24,6 +24,8 @@ MUTATIONS = {
     "ln_var_drop_mean": ("float d = h2f(x[k0]) - mean;", "float d = h2f(x[k0]);"),
     "ln_unbiased_var": ("float var = chunk_tree_sum(x, K, 1, mean) / (float)K;",
                         "float var = chunk_tree_sum(x, K, 1, mean) / (float)(K - 1);"),
+    "ln_one_pass_var": ("float var = chunk_tree_sum(x, K, 1, mean) / (float)K;",
+                        "float var = chunk_tree_sum(x, K, 1, 0.0f) / (float)K - mean * mean;"),
     "ln_tree_skips_pad": ("for (int c = 0; c < n; c += 2 * step) v[c] = v[c] + v[c + step];",
                           "for (int c = 0; c + step < n - 1; c += 2 * step) v[c] = v[c] + v[c + step];"),
     "gemm_reversed_k": ("for (int k = 0; k < K; ++k) s += (int64_t)a[k] * (int64_t)b[k];",

@@ -224,9 +224,12 @@ zq_status zq_gemm_w4a16(const void* X, const uint8_t* Wq4, const float* s_grp, i
  *   8 MiB in device memory that the library declares statically; every GPU
  *   that loads the library holds it until the process exits, and no call of
  *   this function allocates or frees anything.
- *   Limit: when the planned split-K reduction needs more than that, i.e.
- *   splits * T * N int32 partial sums above 8 MiB, the call returns
- *   ZQ_ERR_SHAPE without launching.
+ *   It chooses the same kernel and tiling as zq_gemm_w8a8.
+ *   Limit: when that plan's split-K reduction would need more than the
+ *   array holds (splits * T * N int32 partial sums above 8 MiB), the call
+ *   plans again with as many K splits as fit (one split needs no scratch).
+ *   Only a split count forced through ZQ_OPT_SPLIT_K that does not fit is
+ *   refused: ZQ_ERR_SHAPE, without launching.
  *   The first call on a device looks up the array's device address (with
  *   that device current); make that first call before any stream capture.
  *   All calls on a device share the one array: calls whose work may overlap

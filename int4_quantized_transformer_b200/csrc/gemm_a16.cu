@@ -38,6 +38,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "zq_internal.h"
 #include "zq_ptx.cuh"
@@ -569,21 +570,21 @@ A16Plan plan_a16(int T, int N, int K, int sms, int forced_bn, bool pair) {
 template <class C>
 cudaError_t launch_a16(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& my,
                        const A16Params& p, int grid, cudaStream_t st) {
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];  // per device; a repeated set is harmless
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     e = cudaFuncSetAttribute(gemm_a16_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   if constexpr (C::PAIR) {
     // no more pairs than can be resident at once (a second, serial wave of a
     // persistent grid would only add a tail)
-    static int max_pairs[64] = {};
-    if (dev >= 0 && dev < 64 && max_pairs[dev] == 0) {
+    static std::atomic<int> max_pairs[64];
+    if (dev >= 0 && dev < 64 && max_pairs[dev].load(std::memory_order_acquire) == 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(grid);
       cfg.blockDim = dim3(C::NUM_THREADS);
@@ -600,9 +601,9 @@ cudaError_t launch_a16(const CUtensorMap& mx, const CUtensorMap& mw, const CUten
         cudaGetLastError();
         n = 1 << 20;  // unknown: keep the requested grid
       }
-      max_pairs[dev] = n;
+      max_pairs[dev].store(n, std::memory_order_release);
     }
-    if (dev >= 0 && dev < 64) grid = std::min(grid, 2 * max_pairs[dev]);
+    if (dev >= 0 && dev < 64) grid = std::min(grid, 2 * max_pairs[dev].load());
     return launch_pdl_cluster(gemm_a16_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
                               static_cast<size_t>(C::SMEM_BYTES), st, 2u, mx, mw, my, p);
   }

@@ -43,6 +43,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "zq_internal.h"
@@ -1093,21 +1094,23 @@ template <class C>
 cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUtensorMap& my,
                        const GemmParams& gp, int grid, cudaStream_t st) {
   // grid: CTAs requested; clamped below for CTA pairs
-  static bool attr_set[64] = {};
+  // per device and kernel variant; several host threads may race here, and
+  // setting the attribute twice is harmless
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_i8_kernel<C>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   if constexpr (C::PAIR) {
     // A persistent grid of pairs larger than the number of pairs that can be
     // resident at once would leave a second, serial wave: clamp to it.
-    static int max_pairs[64] = {};
-    if (dev >= 0 && dev < 64 && max_pairs[dev] == 0) {
+    static std::atomic<int> max_pairs[64];
+    if (dev >= 0 && dev < 64 && max_pairs[dev].load(std::memory_order_acquire) == 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(grid);
       cfg.blockDim = dim3(C::NUM_THREADS);
@@ -1124,9 +1127,9 @@ cudaError_t launch_cfg(const CUtensorMap& ma, const CUtensorMap& mw, const CUten
         cudaGetLastError();
         n = 1 << 20;  // unknown: keep the requested grid
       }
-      max_pairs[dev] = n;
+      max_pairs[dev].store(n, std::memory_order_release);
     }
-    if (dev >= 0 && dev < 64) grid = std::min(grid, 2 * max_pairs[dev]);
+    if (dev >= 0 && dev < 64) grid = std::min(grid, 2 * max_pairs[dev].load());
   }
   cudaError_t e =
       C::PAIR ? launch_pdl_cluster(gemm_i8_kernel<C>, dim3(grid), dim3(C::NUM_THREADS),
@@ -1167,9 +1170,11 @@ cudaError_t dispatch_bn(int bn, const CUtensorMap& ma, const CUtensorMap& mw,
   }
 }
 
-zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* Wq,
-                     const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,
-                     int32_t* acc_dbg, zq_stream_t stream) {
+// The checks shared by every GEMM entry point (synchronous, before any
+// launch).
+zq_status check_gemm_args(bool w4, const int8_t* Xq, const float* s_tok, const void* Wq,
+                          const float* s_grp, int g, const void* bias, int T, int N, int K,
+                          const void* Y, const int32_t* acc_dbg) {
   if (T < 0 || N < 8 || N % 8 != 0 || K < 16 || K % 16 != 0 || K > 133136) return ZQ_ERR_SHAPE;
   if (w4 && (K % 32 != 0 || K > 132096)) return ZQ_ERR_SHAPE;
   if (g < 1 || g > N) return ZQ_ERR_SHAPE;
@@ -1178,9 +1183,18 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || (bias && !aligned16(bias)) ||
       (acc_dbg && !aligned16(acc_dbg)))
     return ZQ_ERR_ALIGN;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int sms = num_sms();
+  return ZQ_OK;
+}
 
+// The kernel a call runs: the CUDA-core matrix-vector path, or a tensor-core
+// plan.  forced_split > 0 fixes the number of K splits of a weight-row plan.
+struct Choice {
+  bool gemv = false;
+  Plan plan{};
+};
+
+zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
+  const int sms = num_sms();
   // A handful of tokens: the CUDA-core matrix-vector path (measured faster
   // than the tensor-core tilings up to T = 4 with INT4 weights and up to
   // T = 2 with INT8 ones).  Otherwise weight rows on the MMA M side for small
@@ -1189,35 +1203,51 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   const int forced_path = option(ZQ_OPT_GEMM_PATH);
   if (forced_path == 3 || (forced_path == 0 && T <= gemv_max_tokens(w4))) {
     if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
+    out->gemv = true;
+    return ZQ_OK;
+  }
+  out->gemv = false;
+  if (forced_path == 2 || (forced_path == 0 && use_weight_rows(T, K, w4))) {
+    out->plan = plan_wrows(T, N, K, sms, forced_split, w4);
+    return ZQ_OK;
+  }
+  const int fbn = option(ZQ_OPT_GEMM_BN);
+  if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
+  // CTA pairs need less operand traffic per SM (32 KB instead of 48 KB per
+  // 128-deep K slice) but pay a cross-CTA handshake per stage and per
+  // tile.  Measured on B200 over the layer shapes: pairs of 256 x 256
+  // tiles run ~18% faster per tile when K >= 2048 and ~10% slower at small
+  // K, so the two wave-aware plans are compared with those factors.
+  const int fpair = option(ZQ_OPT_CTA_PAIR);
+  const Plan single = plan_trows(T, N, K, sms, fbn, false);
+  if (fpair == 1) {
+    out->plan = single;
+    return ZQ_OK;
+  }
+  const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true);
+  // INT4: the unpack stage, not the operand feed, bounds the mainloop;
+  // pairs measured slower there, so they are used only when forced.
+  const double f = w4 ? 1e9 : (K >= 2048 ? 0.82 : 1.10);
+  out->plan = (fpair == 2 || pr.cost * f < single.cost) ? pr : single;
+  return ZQ_OK;
+}
+
+// Partial sums a weight-row plan with K splits stores (int32 elements).
+size_t split_partials(const Plan& plan, int T, int N) {
+  return (plan.wrows && plan.splits > 1) ? static_cast<size_t>(plan.splits) * T * N : 0;
+}
+
+// Launches a chosen plan; `ws` receives the split-K partial sums (at least
+// split_partials() elements) when the plan splits K.
+zq_status launch_choice(bool w4, const Choice& ch, const int8_t* Xq, const float* s_tok,
+                        const void* Wq, const float* s_grp, int g, const void* bias, int T, int N,
+                        int K, void* Y, int32_t* acc_dbg, int32_t* ws, cudaStream_t st) {
+  if (ch.gemv)
     return launch_gemv_i8(w4 ? 4 : 8, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg,
                           option(ZQ_OPT_MAX_CTAS), st) == cudaSuccess
                ? ZQ_OK
                : ZQ_ERR_CUDA;
-  }
-  Plan plan;
-  if (forced_path == 2 || (forced_path == 0 && use_weight_rows(T, K, w4))) {
-    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K), w4);
-  } else {
-    const int fbn = option(ZQ_OPT_GEMM_BN);
-    if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
-    // CTA pairs need less operand traffic per SM (32 KB instead of 48 KB per
-    // 128-deep K slice) but pay a cross-CTA handshake per stage and per
-    // tile.  Measured on B200 over the layer shapes: pairs of 256 x 256
-    // tiles run ~18% faster per tile when K >= 2048 and ~10% slower at small
-    // K, so the two wave-aware plans are compared with those factors.
-    const int fpair = option(ZQ_OPT_CTA_PAIR);
-    const Plan single = plan_trows(T, N, K, sms, fbn, false);
-    if (fpair == 1) {
-      plan = single;
-    } else {
-      const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true);
-      // INT4: the unpack stage, not the operand feed, bounds the mainloop;
-      // pairs measured slower there, so they are used only when forced.
-      const double f = w4 ? 1e9 : (K >= 2048 ? 0.82 : 1.10);
-      plan = (fpair == 2 || pr.cost * f < single.cost) ? pr : single;
-    }
-  }
-
+  const Plan& plan = ch.plan;
   int* status = device_status_ptr();
   if (!status) return ZQ_ERR_CUDA;
 
@@ -1227,6 +1257,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   gp.bias = static_cast<const __half*>(bias);
   gp.Y = static_cast<__half*>(Y);
   gp.acc_dbg = acc_dbg;
+  gp.ws = ws;
   gp.status = status;
   gp.T = T;
   gp.N = N;
@@ -1243,12 +1274,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   // weight tile then comes from DRAM once, the activations from L2).
   gp.n_fastest = plan.wrows && plan.n_tiles > 1 &&
                  static_cast<double>(N) * K * (w4 ? 0.5 : 1.0) > static_cast<double>(T) * K;
-  if (plan.wrows && plan.splits > 1) {
-    Workspace* w = nullptr;
-    if (ensure_workspace(static_cast<size_t>(plan.splits) * T * N, &w) != cudaSuccess)
-      return ZQ_ERR_CUDA;
-    gp.ws = w->ws;
-  }
+  if (split_partials(plan, T, N) > 0 && !ws) return ZQ_ERR_CUDA;
 
   // TMA descriptors: int8 activations [T][K]; weights int8 [N][K] (128B
   // swizzle, matching the MMA's K-major layout) or packed int4 [N][K/2]
@@ -1276,6 +1302,7 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   if (!encode_y_map(&my, Y, T, N))
     return ZQ_ERR_CUDA;
 
+  const int sms = num_sms();
   int grid = std::min(plan.units, sms);
   const int cap = option(ZQ_OPT_MAX_CTAS);
   if (cap > 0) grid = std::min(grid, cap);
@@ -1293,8 +1320,27 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   else
     e = w4 ? dispatch_bn<false, true>(plan.bn, ma, mw, my, gp, grid, st)
            : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
-  if (e == cudaSuccess && plan.wrows && plan.splits > 1) e = launch_finalize(gp, st);
+  if (e == cudaSuccess && split_partials(plan, T, N) > 0) e = launch_finalize(gp, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
+
+zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* Wq,
+                     const float* s_grp, int g, const void* bias, int T, int N, int K, void* Y,
+                     int32_t* acc_dbg, zq_stream_t stream) {
+  zq_status rc = check_gemm_args(w4, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg);
+  if (rc != ZQ_OK || T == 0) return rc;
+  Choice ch;
+  rc = choose(w4, T, N, K, option(ZQ_OPT_SPLIT_K), &ch);
+  if (rc != ZQ_OK) return rc;
+  int32_t* ws = nullptr;
+  const size_t partials = ch.gemv ? 0 : split_partials(ch.plan, T, N);
+  if (partials > 0) {
+    Workspace* w = nullptr;
+    if (ensure_workspace(partials, &w) != cudaSuccess) return ZQ_ERR_CUDA;
+    ws = w->ws;
+  }
+  return launch_choice(w4, ch, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg, ws,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -1361,82 +1407,29 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
                                           int N, int K, void* Y, int32_t* acc_dbg,
                                           zq_stream_t stream) {
   using namespace zq;
-  if (T < 0 || N < 8 || N % 8 != 0 || K < 16 || K % 16 != 0 || K > 133136) return ZQ_ERR_SHAPE;
-  if (g < 1 || g > N) return ZQ_ERR_SHAPE;
-  if (T == 0) return ZQ_OK;
-  if (!Xq || !s_tok || !Wq || !s_grp || !Y) return ZQ_ERR_NULL;
-  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || (bias && !aligned16(bias)) ||
-      (acc_dbg && !aligned16(acc_dbg)))
-    return ZQ_ERR_ALIGN;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int sms = num_sms();
-
-  const int forced_path = option(ZQ_OPT_GEMM_PATH);
-  // the matrix-vector path (as in zq_gemm_w8a8) needs no scratch at all
-  if (forced_path == 3 || (forced_path == 0 && T <= gemv_max_tokens(false))) {
-    if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
-    return launch_gemv_i8(8, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg,
-                          option(ZQ_OPT_MAX_CTAS), st) == cudaSuccess
-               ? ZQ_OK
-               : ZQ_ERR_CUDA;
+  zq_status rc = check_gemm_args(false, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg);
+  if (rc != ZQ_OK || T == 0) return rc;
+  // The same choice of kernel and plan as zq_gemm_w8a8.  When its K splits
+  // would need more partial sums than the fixed array holds, plan again with
+  // as many splits as fit (one split needs no scratch at all); only a split
+  // count forced through ZQ_OPT_SPLIT_K that does not fit is refused.
+  const int forced_split = option(ZQ_OPT_SPLIT_K);
+  Choice ch;
+  rc = choose(false, T, N, K, forced_split, &ch);
+  if (rc != ZQ_OK) return rc;
+  if (!ch.gemv && split_partials(ch.plan, T, N) > kNoAllocPartialInts) {
+    if (forced_split > 0) return ZQ_ERR_SHAPE;
+    const size_t fit = kNoAllocPartialInts / (static_cast<size_t>(T) * N);
+    rc = choose(false, T, N, K, static_cast<int>(std::max<size_t>(1, std::min<size_t>(fit, 32))),
+                &ch);
+    if (rc != ZQ_OK) return rc;
+    if (split_partials(ch.plan, T, N) > kNoAllocPartialInts) return ZQ_ERR_SHAPE;
   }
-  Plan plan;
-  if (forced_path == 2 || (forced_path == 0 && T <= 256)) {
-    plan = plan_wrows(T, N, K, sms, option(ZQ_OPT_SPLIT_K), false);
-  } else {
-    const int fbn = option(ZQ_OPT_GEMM_BN);
-    if (fbn && fbn != 128 && fbn != 192 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
-    plan = plan_trows(T, N, K, sms, fbn, false);
-  }
-
-  int* status = device_status_ptr();
-  if (!status) return ZQ_ERR_CUDA;
-
-  GemmParams gp{};
-  gp.s_tok = s_tok;
-  gp.s_grp = s_grp;
-  gp.bias = static_cast<const __half*>(bias);
-  gp.Y = static_cast<__half*>(Y);
-  gp.acc_dbg = acc_dbg;
-  gp.status = status;
-  gp.T = T;
-  gp.N = N;
-  gp.K = K;
-  gp.g = g;
-  gp.m_tiles = plan.m_tiles;
-  gp.n_tiles = plan.n_tiles;
-  gp.k_blocks = plan.k_blocks;
-  gp.splits = plan.splits;
-  gp.kb_per_split = plan.kb_per_split;
-  gp.num_units = plan.units;
-  gp.n_fastest = plan.wrows && plan.n_tiles > 1 &&
-                 static_cast<double>(N) * K > static_cast<double>(T) * K;
-  if (plan.wrows && plan.splits > 1) {
-    const size_t partial = static_cast<size_t>(plan.splits) * T * N;
-    if (partial > kNoAllocPartialInts) return ZQ_ERR_SHAPE;
-    int32_t* scratch = nullptr;
+  int32_t* scratch = nullptr;
+  if (!ch.gemv && split_partials(ch.plan, T, N) > 0) {
     if (noalloc_scratch(&scratch) != cudaSuccess) return ZQ_ERR_CUDA;
     // every partial sum the finalisation reads is written by this call
-    gp.ws = scratch;
   }
-
-  const int act_rows = plan.wrows ? plan.bn : BM;
-  const int w_rows = plan.wrows ? BM : plan.bn;
-  CUtensorMap ma, mw, my;
-  if (!encode_tma_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, T, K, BK, act_rows,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
-    return ZQ_ERR_CUDA;
-  if (!encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, K, N, K, BK, w_rows,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
-    return ZQ_ERR_CUDA;
-  if (!encode_y_map(&my, Y, T, N))
-    return ZQ_ERR_CUDA;
-
-  int grid = std::min(plan.units, sms);
-  const int cap = option(ZQ_OPT_MAX_CTAS);
-  if (cap > 0) grid = std::min(grid, cap);
-  cudaError_t e = plan.wrows ? dispatch_bn<true, false>(plan.bn, ma, mw, my, gp, grid, st)
-                             : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
-  if (e == cudaSuccess && plan.wrows && plan.splits > 1) e = launch_finalize(gp, st);
-  return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+  return launch_choice(false, ch, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg, scratch,
+                       reinterpret_cast<cudaStream_t>(stream));
 }

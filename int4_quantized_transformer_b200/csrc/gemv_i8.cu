@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "zq_internal.h"
 #include "zq_ptx.cuh"
@@ -184,10 +185,10 @@ template <int BITS, int TT>
 cudaError_t launch_tt(const int8_t* Xq, const float* s_tok, const void* W, const float* s_grp,
                       int g, const void* bias, int T, int N, int K, void* Y, int32_t* acc_dbg,
                       int max_ctas, cudaStream_t st) {
-  static int resident[64] = {};
+  static std::atomic<int> resident[64];  // per device; a repeated query is harmless
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && resident[dev] == 0) {
+  if (dev >= 0 && dev < 64 && resident[dev].load(std::memory_order_acquire) == 0) {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_i8_kernel<BITS, TT>,
                                                       kGemvThreads, 0) != cudaSuccess ||
@@ -195,9 +196,9 @@ cudaError_t launch_tt(const int8_t* Xq, const float* s_tok, const void* W, const
       cudaGetLastError();
       per_sm = 1;
     }
-    resident[dev] = per_sm;
+    resident[dev].store(per_sm, std::memory_order_release);
   }
-  const int per_sm = (dev >= 0 && dev < 64) ? resident[dev] : 1;
+  const int per_sm = (dev >= 0 && dev < 64) ? resident[dev].load() : 1;
   constexpr int kRows = GemvShape<TT>::ROWS;
   constexpr int round = 32 * GemvShape<TT>::UNROLL;
   const int chunks = K / (BITS == 4 ? 32 : 16);

@@ -93,3 +93,66 @@ def test_noalloc_forced_splits_and_oversize_rejected(zq):
                                            torch.cuda.current_stream().cuda_stream)
     assert rc == zq.ZQ_ERR_SHAPE
     assert zq.device_status()[0] == zq.ZQ_OK
+
+
+def test_noalloc_replans_splits_that_do_not_fit(zq):
+    # The automatic plan for 256 tokens x 4096 outputs x K = 16384 splits K
+    # four ways (16 MiB of partial sums); the allocation-free call plans again
+    # with as many splits as its fixed array holds and gives the same result.
+    ops = _operands(zq, 256, 4096, 16384, 64, 11)
+    y_ref, acc_ref = _call(zq, "zq_gemm_w8a8", *ops)
+    for _ in range(2):
+        y, acc = _call(zq, "zq_gemm_w8a8_noalloc", *ops)
+        _assert_same(y, acc, y_ref, acc_ref)
+    assert zq.device_status()[0] == zq.ZQ_OK
+
+
+_FRESH = r"""
+import sys, torch
+sys.path.insert(0, {root!r})
+from int4_quantized_transformer_b200 import zq
+T, N, K, g = 64, 4096, 8192, 64
+Xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, device="cuda")
+st = torch.rand(T, device="cuda")
+Wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device="cuda")
+sg = torch.rand(g, device="cuda")
+outs = [torch.empty((T, N), dtype=torch.float16, device="cuda") for _ in range(3)]
+s = torch.cuda.current_stream().cuda_stream
+
+def call(name, Y):
+    rc = getattr(zq.lib(), name)(Xq.data_ptr(), st.data_ptr(), Wq.data_ptr(), sg.data_ptr(), g,
+                                 None, T, N, K, Y.data_ptr(), None, s)
+    assert rc == zq.ZQ_OK, zq.status_str(rc)
+    torch.cuda.synchronize()
+
+torch.cuda.synchronize()
+with zq.options(path=2, split_k=4):  # 4 x 64 x 4096 int32 partial sums = 4 MiB
+    free0 = torch.cuda.mem_get_info()[0]
+    call("zq_gemm_w8a8_noalloc", outs[0])
+    call("zq_gemm_w8a8_noalloc", outs[1])
+    free1 = torch.cuda.mem_get_info()[0]
+    call("zq_gemm_w8a8", outs[2])  # the allocating entry point: its workspace shows
+    free2 = torch.cuda.mem_get_info()[0]
+assert torch.equal(outs[0], outs[2]) and torch.equal(outs[1], outs[2])
+print(free0, free1, free2)
+"""
+
+
+def test_noalloc_first_call_in_a_fresh_process_allocates_nothing():
+    """In a fresh process whose kernels are all loaded up front, the first
+    GEMM call of the library is an allocation-free call at a split-K shape:
+    the device's free memory is the same before and after it (and after a
+    second one), while the allocating entry point's split-K workspace, 4 MiB
+    here, does show up afterwards."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_MODULE_LOADING="EAGER")
+    out = subprocess.run([sys.executable, "-c", _FRESH.format(root=root)], env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-3000:]
+    free0, free1, free2 = (int(v) for v in out.stdout.split()[-3:])
+    assert free1 == free0, (free0, free1)
+    assert free2 <= free1 - 4 * 1024 * 1024, (free1, free2)

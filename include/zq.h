@@ -147,9 +147,12 @@ zq_status zq_static_quant(const void* X, int T, int K, float amax, int8_t* Xq, f
  * Runs on tcgen05 tensor cores, except for T <= 2 (INT8) or T <= 4 (INT4
  * weights), a memory-bound matrix-vector product that runs on CUDA cores
  * (dp4a, exact int32).  Small T (weight-streaming) tensor-core shapes split
- * K across SMs: the exact int32 partial sums go to a library-owned workspace
- * and a second kernel on the same stream adds them and dequantizes; calls
- * that use the workspace on different streams must not overlap.
+ * K across SMs: the exact int32 partial sums go to the library workspace
+ * and a second kernel on the same stream adds them and dequantizes.
+ * The library workspace is one device buffer per device, grown with
+ * cudaMalloc the first time a call needs more than it holds (see
+ * zq_workspace_reserve to size it up front); calls that use it on
+ * different streams must not overlap.
  * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
  * 16 <= K <= 133136, K % 16 == 0 (so that 127*127*K < 2^31), 1 <= g <= N,
  * pointers 16-byte aligned.
@@ -161,10 +164,14 @@ zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
 /*
  * zq_gemm_w4a8 -- as zq_gemm_w8a8 with INT4 weights (Sec. 3.4 "Which weights
  * get INT4": FFN weights in INT4).  Wq4 is uint8 [N][K/2] in the layout of
- * zq_quantize_weights_groupwise(bits=4); the kernel unpacks the nibbles to
- * int8 before each tensor-core MMA: in shared memory for token-row tiles,
- * in tensor memory (the MMA's A operand) for weight-row tiles, which this
- * function uses up to T = 128 and for T >= 1024 when K >= 2048.
+ * zq_quantize_weights_groupwise(bits=4).  The nibbles are widened to int8
+ * codes before the tensor-core MMAs read them:
+ *   - T >= 1024 (prefill): once per call, by an HBM-bound pass into the
+ *     library workspace (N*K bytes), which the INT8 GEMM then reads;
+ *   - 128 < T < 1024: in shared memory, inside each token-row tile;
+ *   - 4 < T <= 128: in tensor memory (the MMA's A operand), inside each
+ *     weight-row tile;
+ *   - T <= 4: in registers, on the CUDA-core matrix-vector path.
  * Requirements as zq_gemm_w8a8, plus K % 32 == 0 and K <= 132096.
  */
 zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
@@ -256,7 +263,10 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  *                      2 = weight rows on the MMA M side (weight streaming),
  *                      3 = CUDA-core matrix-vector product (T <= 4, else
  *                          ZQ_ERR_UNSUPPORTED); automatic at T <= 4 with
- *                          INT4 weights and at T <= 2 with INT8 ones.
+ *                          INT4 weights and at T <= 2 with INT8 ones;
+ *                      4 = INT4 weights widened into the workspace, then
+ *                          the INT8 GEMM (zq_gemm_w4a8 only, else
+ *                          ZQ_ERR_UNSUPPORTED); automatic at T >= 1024.
  *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256);
  *                      the FP16-activation GEMMs accept 128 or 256 (other
  *                      values: ZQ_ERR_UNSUPPORTED) and ignore the path.
@@ -275,6 +285,17 @@ typedef enum {
 } zq_option;
 zq_status zq_set_option(int key, int value);
 int zq_get_option(int key);
+
+/*
+ * zq_workspace_reserve -- grow the library workspace of the current device
+ * to at least `bytes` now (cudaMalloc; nothing happens if it is that large
+ * already), so that later GEMM calls of up to that need allocate nothing.
+ * The need of a call: 4 * splits * T * N bytes for a split-K weight-streaming
+ * plan, plus N * K bytes (rounded up to 256) when zq_gemm_w4a8 widens its
+ * codes (T >= 1024, or ZQ_OPT_GEMM_PATH = 4).  Synchronous; call it
+ * outside stream capture.  Returns ZQ_ERR_CUDA if the allocation fails.
+ */
+zq_status zq_workspace_reserve(unsigned long long bytes);
 
 /*
  * zq_launch_count -- number of kernel launches this library has issued in

@@ -945,6 +945,43 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// INT4 weights for prefill-sized token counts: the packed codes are widened
+// once per call to int8 codes in a workspace, [N][K] in k order, and the
+// INT8 GEMM reads them from there.  Each weight tile is then widened once
+// instead of once per token tile, and the GEMM's shared memory carries only
+// the TMA copies and the MMA operand reads (the widening inside the tiles,
+// through shared memory or into tensor memory, competes with both).  The
+// pass is HBM-bound: N*K/2 bytes read and N*K written.
+//
+// Of each 32-bit word of packed codes (eight consecutive k), byte i holds
+// k = i in its low nibble and k = 4 + i in its high nibble; a nibble n is the
+// two's-complement code n - 16 * (n >= 8), i.e. the byte n | 0xF0 when bit 3
+// is set (the mask times 0x1E sets the four high bits of exactly those
+// bytes, with no carry between bytes).
+__device__ __forceinline__ uint32_t sext_nibbles(uint32_t n) {
+  return n | ((n & 0x08080808u) * 0x1Eu);
+}
+
+__global__ void __launch_bounds__(256)
+    widen_w4_kernel(const uint4* __restrict__ packed, uint4* __restrict__ wide, size_t n16) {
+  // the packed codes may be written by the previous kernel of the stream
+  grid_dependency_wait();
+  grid_launch_dependents();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 w = __ldcs(packed + i);  // 32 codes: k = 32i .. 32i + 31 of one row
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t out[8];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      out[2 * m] = sext_nibbles(in[m] & 0x0F0F0F0Fu);             // k = 8m .. 8m + 3
+      out[2 * m + 1] = sext_nibbles((in[m] >> 4) & 0x0F0F0F0Fu);  // k = 8m + 4 .. 8m + 7
+    }
+    wide[2 * i] = make_uint4(out[0], out[1], out[2], out[3]);
+    wide[2 * i + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
+
 // ------------------------------------------------------------------ host
 
 struct Workspace {
@@ -1000,16 +1037,14 @@ int gemv_max_tokens(bool w4) { return w4 ? kGemvMaxTokens : 2; }
 
 // The automatic choice of weight rows on the MMA M side (above the
 // matrix-vector range).  INT8 weights: up to 256 tokens (weight streaming).
-// INT4 weights: up to 128 tokens, and also for prefill-sized token counts
-// with long rows (T >= 1024, K >= 2048), where widening the weights into
-// tensor memory beats the token-row tiles' widening through shared memory
-// (measured on B200: GPT-NeoX FFN1/FFN2 at T = 4096 697/767 us instead of
-// 772/873 us, GPT-3 350M FFN2 at T = 16384 87 us instead of 117 us); with
-// short rows (K = 1024) or few tokens the token-row tiles stay ahead, since
-// each weight-row tile re-reads its whole activation block.
+// INT4 weights: up to 128 tokens, where the widened weights live in tensor
+// memory next to the accumulators; from 1024 tokens the widening pass and
+// the INT8 GEMM take over (kWidenMinTokens), and in between the token-row
+// tiles widen the weights through shared memory.
 bool use_weight_rows(int T, int K, bool w4) {
+  (void)K;
   if (!w4) return T <= 256;
-  return T <= 128 || (T >= 1024 && K >= 2048);
+  return T <= 128;
 }
 
 // fp16 output [T][N]: 32 x 32 boxes written by the epilogue warps
@@ -1190,8 +1225,14 @@ zq_status check_gemm_args(bool w4, const int8_t* Xq, const float* s_tok, const v
 // plan.  forced_split > 0 fixes the number of K splits of a weight-row plan.
 struct Choice {
   bool gemv = false;
+  bool widen = false;  // INT4 weights widened into the workspace, then the INT8 plan
   Plan plan{};
 };
+
+// INT4 weights at prefill-sized token counts take the widening pass and the
+// INT8 GEMM (widen_w4_kernel): from 1024 tokens up, the pass costs well
+// under a tenth of the GEMM.
+constexpr int kWidenMinTokens = 1024;
 
 zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
   const int sms = num_sms();
@@ -1200,7 +1241,15 @@ zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
   // T = 2 with INT8 ones).  Otherwise weight rows on the MMA M side for small
   // token counts (weight streaming), token rows beyond; tests and benchmarks
   // may force any of them.
-  const int forced_path = option(ZQ_OPT_GEMM_PATH);
+  int forced_path = option(ZQ_OPT_GEMM_PATH);
+  out->widen = false;
+  if (forced_path == 4 && !w4) return ZQ_ERR_UNSUPPORTED;
+  if (w4 && (forced_path == 4 || (forced_path == 0 && T >= kWidenMinTokens))) {
+    // the INT8 GEMM on the widened codes, planned as for INT8 weights
+    out->widen = true;
+    w4 = false;
+    forced_path = 0;
+  }
   if (forced_path == 3 || (forced_path == 0 && T <= gemv_max_tokens(w4))) {
     if (T > kGemvMaxTokens) return ZQ_ERR_UNSUPPORTED;
     out->gemv = true;
@@ -1332,19 +1381,38 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   Choice ch;
   rc = choose(w4, T, N, K, option(ZQ_OPT_SPLIT_K), &ch);
   if (rc != ZQ_OK) return rc;
-  int32_t* ws = nullptr;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // One library workspace per device: the widened INT4 codes (N*K bytes,
+  // rounded up to 256 bytes) first, when the call widens, then the split-K
+  // partial sums, when its plan splits K.
   const size_t partials = ch.gemv ? 0 : split_partials(ch.plan, T, N);
-  if (partials > 0) {
+  const size_t wide_ints = ch.widen ? (static_cast<size_t>(N) * K + 255) / 256 * 64 : 0;
+  int32_t* ws = nullptr;
+  if (partials > 0 || wide_ints > 0) {
     Workspace* w = nullptr;
-    if (ensure_workspace(partials, &w) != cudaSuccess) return ZQ_ERR_CUDA;
+    if (ensure_workspace(wide_ints + partials, &w) != cudaSuccess) return ZQ_ERR_CUDA;
     ws = w->ws;
   }
-  return launch_choice(w4, ch, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg, ws,
-                       reinterpret_cast<cudaStream_t>(stream));
+  if (ch.widen) {
+    const size_t n16 = static_cast<size_t>(N) * (K / 2) / 16;
+    const int blocks = static_cast<int>(std::min<size_t>((n16 + 255) / 256, 8 * num_sms()));
+    if (launch_pdl(widen_w4_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, st,
+                   static_cast<const uint4*>(Wq), reinterpret_cast<uint4*>(ws), n16) != cudaSuccess)
+      return ZQ_ERR_CUDA;
+    return launch_choice(false, ch, Xq, s_tok, ws, s_grp, g, bias, T, N, K, Y, acc_dbg,
+                         partials > 0 ? ws + wide_ints : nullptr, st);
+  }
+  return launch_choice(w4, ch, Xq, s_tok, Wq, s_grp, g, bias, T, N, K, Y, acc_dbg, ws, st);
 }
 
 }  // namespace
 }  // namespace zq
+
+extern "C" zq_status zq_workspace_reserve(unsigned long long bytes) {
+  zq::Workspace* w = nullptr;
+  if (bytes == 0) return ZQ_OK;
+  return zq::ensure_workspace((bytes + 3) / 4, &w) == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
 
 extern "C" zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
                                   const float* s_grp, int g, const void* bias, int T, int N,

@@ -18,6 +18,8 @@
 // with respect to the op-by-op definition in include/zq.h.
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "zq_internal.h"
 #include "zq_ptx.cuh"
 
@@ -144,12 +146,67 @@ __device__ __forceinline__ float row_tree_sum(float (&cs)[VPT], float* red, int 
   return v[0];
 }
 
+// Packed and mixed-precision fp32 arithmetic of sm_100 (PTX ISA 8.6): two
+// independent IEEE round-to-nearest operations per instruction (f32x2), and
+// an add or subtract whose first operand is fp16 (converted exactly, then
+// one rounding).  They give the same bits as the scalar operations, with
+// fewer instructions per element.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+// f32(h) + c and f32(h) - c, one rounding each
+__device__ __forceinline__ float add_h(uint16_t h, float c) {
+  float r;
+  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(r) : "h"(h), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float sub_h(uint16_t h, float c) {
+  float r;
+  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(r) : "h"(h), "f"(c));
+  return r;
+}
+__device__ __forceinline__ void halves(uint32_t w, uint16_t& lo, uint16_t& hi) {
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
+}
+// running max of |.| over packed fp16 pairs (the sign of the result is
+// meaningless; its magnitude is max(|a|, |b|) per half)
+__device__ __forceinline__ uint32_t hmax_abs2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// LayerNorm gamma/beta are kept as fp32 in shared memory (converted once per
+// CTA) when both fit in this many bytes; longer rows convert per row.
+constexpr int kGammaBetaSmemMax = 64 * 1024;
+
 // W warps per row, VPT 16-byte vectors (8 halves) per thread.  Blocks hold
 // RPB = max(1, 8/W) rows; every thread runs the same number of row
-// iterations so block-wide barriers stay uniform.  gamma/beta are re-read
-// per row (they stay in L1) to keep registers low and occupancy high.
+// iterations so block-wide barriers stay uniform.  The loads of a thread's
+// next row are issued before the current row is reduced, so their latency
+// overlaps its arithmetic.
 template <int W, int VPT>
-__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 32) : 8) / 2)
+__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
     ln_quant_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
                     const __half* __restrict__ beta, const __half* __restrict__ act_bias,
                     int act, float static_amax, int T, int K, float eps,
@@ -161,6 +218,7 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
   __shared__ float red1[RPB][NBLK];  // block sums of x (W > 1)
   __shared__ float red2[RPB][NBLK];  // block sums of (x - mean)^2 (W > 1)
   __shared__ float red_m[RPB][W];
+  extern __shared__ float4 gb_smem[];  // fp32 gamma [K], then beta [K] (when they fit)
 
   const int slot = threadIdx.x / RT;
   const int j = threadIdx.x % RT;
@@ -168,23 +226,49 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
   const int lane = threadIdx.x & 31;
   const int nvec = K / 8;
   const bool ln = gamma != nullptr;
+  const bool gb_smem_ok = ln && 8 * K <= kGammaBetaSmemMax;
+  const float* g_s = reinterpret_cast<const float*>(gb_smem);
+  const float* b_s = g_s + K;
   grid_dependency_wait();
   grid_launch_dependents();
+  if (gb_smem_ok) {
+    float* gs = reinterpret_cast<float*>(gb_smem);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
+      const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v) : make_uint4(0, 0, 0, 0);
+      const __half2* gh = reinterpret_cast<const __half2*>(&g4);
+      const __half2* bh = reinterpret_cast<const __half2*>(&b4);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 gf = __half22float2(gh[e]);
+        const float2 bf = __half22float2(bh[e]);
+        gs[8 * v + 2 * e] = gf.x;
+        gs[8 * v + 2 * e + 1] = gf.y;
+        gs[K + 8 * v + 2 * e] = bf.x;
+        gs[K + 8 * v + 2 * e + 1] = bf.y;
+      }
+    }
+    __syncthreads();
+  }
 
   const int rows_per_iter = gridDim.x * RPB;
   const int iters = (T + rows_per_iter - 1) / rows_per_iter;
+  auto load_row = [&](uint4 (&dst)[VPT], int row) {
+    const __half* xr = X + static_cast<size_t>(row) * K;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = j + i * RT;
+      dst[i] = make_uint4(0, 0, 0, 0);
+      if (row < T && v < nvec) dst[i] = __ldcs(reinterpret_cast<const uint4*>(xr) + v);
+    }
+  };
+  uint4 x4[VPT];
+  load_row(x4, blockIdx.x * RPB + slot);
   for (int it = 0; it < iters; ++it) {
     const int row = (it * gridDim.x + blockIdx.x) * RPB + slot;
     const bool valid = row < T;
-    const __half* xr = X + static_cast<size_t>(row) * K;
-
-    uint4 x4[VPT];
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      int v = j + i * RT;
-      x4[i] = make_uint4(0, 0, 0, 0);
-      if (valid && v < nvec) x4[i] = __ldcs(reinterpret_cast<const uint4*>(xr) + v);
-    }
+    uint4 n4[VPT];
+    if (it + 1 < iters) load_row(n4, ((it + 1) * gridDim.x + blockIdx.x) * RPB + slot);
 
     if (act >= 0) {
       // the producer of the activation, fused: bias-add (act = 0) or
@@ -217,79 +301,121 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
     }
 
     if (ln) {
-      // mean: chunk sums of x in order, then the pairwise tree
+      // mean: each 8-element chunk summed in index order (the first element
+      // plus -0 is the element itself, exactly), then the pairwise tree
       float cs[VPT];
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
-        const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
-        const float2 f0 = __half22float2(h[0]);
-        float acc = __fadd_rn(f0.x, f0.y);
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
+        float acc = -0.0f;
 #pragma unroll
-        for (int e = 1; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          acc = __fadd_rn(__fadd_rn(acc, f.x), f.y);
+        for (int e = 0; e < 4; ++e) {
+          uint16_t lo, hi;
+          halves(w[e], lo, hi);
+          acc = add_h(hi, add_h(lo, acc));
         }
         cs[i] = acc;  // zero for chunks past the row (x4 is zero there)
       }
       const float mean = __fdiv_rn(row_tree_sum<W, VPT>(cs, red1[slot], lane, warp_in_row),
                                    static_cast<float>(K));
-      // biased variance: chunk sums of (x - mean)^2 (first square, then
-      // fused multiply-adds), then the same tree
+      // deviations x - mean (kept for the normalisation), then the biased
+      // variance: per chunk the first square, then fused multiply-adds in
+      // index order, two chunks at a time in the two halves of f32x2
+      float d[VPT][8];
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
-        const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
-        const float2 f0 = __half22float2(h[0]);
-        const float d0 = __fsub_rn(f0.x, mean);
-        const float d1 = __fsub_rn(f0.y, mean);
-        float acc = __fmaf_rn(d1, d1, __fmul_rn(d0, d0));
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
 #pragma unroll
-        for (int e = 1; e < 4; ++e) {
-          const float2 f = __half22float2(h[e]);
-          const float da = __fsub_rn(f.x, mean);
-          const float db = __fsub_rn(f.y, mean);
-          acc = __fmaf_rn(db, db, __fmaf_rn(da, da, acc));
+        for (int e = 0; e < 4; ++e) {
+          uint16_t lo, hi;
+          halves(w[e], lo, hi);
+          d[i][2 * e] = sub_h(lo, mean);
+          d[i][2 * e + 1] = sub_h(hi, mean);
         }
-        cs[i] = (j + i * RT < nvec) ? acc : 0.0f;  // padding chunks are zero
       }
+#pragma unroll
+      for (int i = 0; i + 1 < VPT; i += 2) {
+        uint64_t q = f2_pack(d[i][0], d[i + 1][0]);
+        q = f2_mul(q, q);
+#pragma unroll
+        for (int e = 1; e < 8; ++e) {
+          const uint64_t de = f2_pack(d[i][e], d[i + 1][e]);
+          q = f2_fma(de, de, q);
+        }
+        f2_unpack(q, cs[i], cs[i + 1]);
+      }
+      if (VPT % 2) {
+        float acc = __fmul_rn(d[VPT - 1][0], d[VPT - 1][0]);
+#pragma unroll
+        for (int e = 1; e < 8; ++e) acc = __fmaf_rn(d[VPT - 1][e], d[VPT - 1][e], acc);
+        cs[VPT - 1] = acc;
+      }
+#pragma unroll
+      for (int i = 0; i < VPT; ++i)
+        if (j + i * RT >= nvec) cs[i] = 0.0f;  // padding chunks are zero
       const float var = __fdiv_rn(row_tree_sum<W, VPT>(cs, red2[slot], lane, warp_in_row),
                                   static_cast<float>(K));
       const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
+      const uint64_t rstd2 = f2_pack(rstd, rstd);
+      // y = fp16(((x - mean) * rstd) * gamma + beta), each step rounded once
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         const int v = j + i * RT;
         if (v < nvec) {
-          const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
-          const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v)
-                                : make_uint4(0, 0, 0, 0);
+          float g[8], b[8];
+          if (gb_smem_ok) {
+            const float4* gp = reinterpret_cast<const float4*>(g_s + 8 * v);
+            const float4* bp = reinterpret_cast<const float4*>(b_s + 8 * v);
+            const float4 g0 = gp[0], g1 = gp[1], b0 = bp[0], b1 = bp[1];
+            g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
+            g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
+            b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
+            b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+          } else {
+            const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
+            const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v)
+                                  : make_uint4(0, 0, 0, 0);
+            const __half2* gh = reinterpret_cast<const __half2*>(&g4);
+            const __half2* bh = reinterpret_cast<const __half2*>(&b4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 gf = __half22float2(gh[e]);
+              const float2 bf = __half22float2(bh[e]);
+              g[2 * e] = gf.x;
+              g[2 * e + 1] = gf.y;
+              b[2 * e] = bf.x;
+              b[2 * e + 1] = bf.y;
+            }
+          }
           __half2* h = reinterpret_cast<__half2*>(&x4[i]);
-          const __half2* gm = reinterpret_cast<const __half2*>(&g4);
-          const __half2* bt = reinterpret_cast<const __half2*>(&b4);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 xf = __half22float2(h[e]);
-            const float2 gf = __half22float2(gm[e]);
-            const float2 bf = __half22float2(bt[e]);
-            const float y0 = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(xf.x, mean), rstd), gf.x), bf.x);
-            const float y1 = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(xf.y, mean), rstd), gf.y), bf.y);
-            h[e] = __halves2half2(__float2half_rn(y0), __float2half_rn(y1));
+            uint64_t t = f2_mul(f2_pack(d[i][2 * e], d[i][2 * e + 1]), rstd2);
+            t = f2_mul(t, f2_pack(g[2 * e], g[2 * e + 1]));
+            t = f2_add(t, f2_pack(b[2 * e], b[2 * e + 1]));
+            float y0, y1;
+            f2_unpack(t, y0, y1);
+            h[e] = __floats2half2_rn(y0, y1);
           }
         }
       }
     }
 
-    __half2 m2 = __float2half2_rn(0.0f);
+    // absmax of the fp16 row (padding vectors are zero)
+    uint32_t m2 = 0u;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const __half2* h = reinterpret_cast<const __half2*>(&x4[i]);
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h[e]));
+      for (int e = 0; e < 4; ++e) m2 = hmax_abs2(m2, w[e]);
     }
     // static quantization: one calibrated range for every token (codes may
     // then exceed the range and are clamped), no per-row reduction
     const bool is_static = static_amax >= 0.0f;  // uniform over the grid
     float amax = static_amax;
     if (!is_static) {
-      amax = warp_max(fmaxf(__low2float(m2), __high2float(m2)));
+      const float2 mf = __half22float2(*reinterpret_cast<const __half2*>(&m2));
+      amax = warp_max(fmaxf(fabsf(mf.x), fabsf(mf.y)));
       if (W > 1) {
         if (lane == 0) red_m[slot][warp_in_row] = amax;
         __syncthreads();
@@ -299,6 +425,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
       }
     }
     const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const uint64_t inv2 = f2_pack(inv, inv);
+    const uint64_t magic2 = f2_pack(12582912.0f, 12582912.0f);
     if (valid) {
       if (j == 0) s_tok[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
       int8_t* qr = Xq + static_cast<size_t>(row) * K;
@@ -311,8 +439,17 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __half22float2(h[e]);
-            c[2 * e] = is_static ? quant_code(f.x, inv, 127.0f) : token_code(f.x, inv);
-            c[2 * e + 1] = is_static ? quant_code(f.y, inv, 127.0f) : token_code(f.y, inv);
+            if (is_static) {
+              c[2 * e] = quant_code(f.x, inv, 127.0f);
+              c[2 * e + 1] = quant_code(f.y, inv, 127.0f);
+            } else {
+              // rne(y * inv) in the low byte: the product, then + 1.5 * 2^23
+              const uint64_t t = f2_add(f2_mul(f2_pack(f.x, f.y), inv2), magic2);
+              float a, b;
+              f2_unpack(t, a, b);
+              c[2 * e] = __float_as_uint(a);
+              c[2 * e + 1] = __float_as_uint(b);
+            }
           }
           uint2 out;
           out.x = pack4(c[0], c[1], c[2], c[3]);
@@ -322,6 +459,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
         }
       }
     }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) x4[i] = n4[i];
   }
 }
 
@@ -331,16 +470,29 @@ cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, const _
                       cudaStream_t st) {
   constexpr int RPB = W >= 8 ? 1 : 8 / W;
   constexpr int threads = RPB * 32 * W;
+  const size_t smem = (g && 8 * K <= kGammaBetaSmemMax) ? static_cast<size_t>(8) * K : 0;
+  // per device; several host threads may race here, and a repeated set is
+  // harmless
+  static std::atomic<bool> attr_set[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(ln_quant_kernel<W, VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGammaBetaSmemMax);
+    if (e != cudaSuccess) return e;
+    attr_set[dev].store(true, std::memory_order_release);
+  }
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &per_sm, ln_quant_kernel<W, VPT>, threads, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_quant_kernel<W, VPT>, threads,
+                                                    smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   int need = (T + RPB - 1) / RPB;
   int grid = num_sms() * per_sm;
   if (grid > need) grid = need;
-  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), 0, st, X, g, b, ab, act, sa,
-                 T, K, eps, Xq, s, Y);
+  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), smem, st, X, g, b, ab, act,
+                 sa, T, K, eps, Xq, s, Y);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -126,7 +126,7 @@ int zq_abi_version(void) { return 104; }
 zq_status zq_set_option(int key, int value) {
   if (key < ZQ_OPT_GEMM_PATH || key > ZQ_OPT_CTA_PAIR) return ZQ_ERR_UNSUPPORTED;
   if (value < 0) return ZQ_ERR_SHAPE;
-  if (key == ZQ_OPT_GEMM_PATH && value > 3) return ZQ_ERR_SHAPE;
+  if (key == ZQ_OPT_GEMM_PATH && value > 4) return ZQ_ERR_SHAPE;
   if (key == ZQ_OPT_CTA_PAIR && value > 2) return ZQ_ERR_SHAPE;
   if (key == ZQ_OPT_GEMM_BN && value != 0 && (value % 16 != 0 || value > 256)) return ZQ_ERR_SHAPE;
   g_opts[key].store(value, std::memory_order_relaxed);

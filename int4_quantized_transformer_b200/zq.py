@@ -24,7 +24,7 @@ EXPORTS = (
     "zq_status_str", "zq_abi_version", "zq_quantize_weights_groupwise", "zq_ln_quant",
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
     "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant", "zq_static_quant",
-    "zq_gemm_w8a16", "zq_gemm_w4a16", "zq_launch_count",
+    "zq_gemm_w8a16", "zq_gemm_w4a16", "zq_launch_count", "zq_workspace_reserve",
 )
 
 
@@ -57,6 +57,7 @@ def _load():
         "zq_gemm_w8a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
         "zq_gemm_w4a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
         "zq_launch_count": ([], ctypes.c_ulonglong),
+        "zq_workspace_reserve": ([ctypes.c_ulonglong], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -102,6 +103,12 @@ def _dev(t: torch.Tensor | None, dtype, shape, name: str):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def workspace_reserve(nbytes: int):
+    """Grow the library workspace of the current device to nbytes now
+    (zq_workspace_reserve)."""
+    _check(_lib.zq_workspace_reserve(int(nbytes)), "zq_workspace_reserve")
 
 
 def launch_count() -> int:

@@ -55,7 +55,7 @@ def test_status_strings_and_version(zq):
 def test_options_validate(zq):
     L = zq.lib()
     assert L.zq_set_option(99, 1) == zq.ZQ_ERR_UNSUPPORTED
-    assert L.zq_set_option(zq.OPT_GEMM_PATH, 4) == zq.ZQ_ERR_SHAPE
+    assert L.zq_set_option(zq.OPT_GEMM_PATH, 5) == zq.ZQ_ERR_SHAPE
     assert L.zq_set_option(zq.OPT_CTA_PAIR, 3) == zq.ZQ_ERR_SHAPE
     assert L.zq_set_option(zq.OPT_GEMM_BN, 100) == zq.ZQ_ERR_SHAPE
     assert L.zq_set_option(zq.OPT_SPLIT_K, -1) == zq.ZQ_ERR_SHAPE

@@ -189,10 +189,33 @@ def test_gemm_auto(zq, bits, T, N, K, g):
                                      (2048, 256, 3072, 4), (1024, 1024, 1024, 16)])
 def test_gemm_w4_tiling_choices(zq, T, N, K, g):
     """INT4 weights choose weight-row tiles (widened weights in TMEM) up to
-    T = 128 and for T >= 1024 with K >= 2048, token-row tiles otherwise; both
-    sides of each boundary, and the forced alternative, match the oracle."""
+    T = 128, token-row tiles up to 1024 tokens and the widening pass with the
+    INT8 GEMM from there; both sides of each boundary, and the forced
+    weight-row alternative, match the oracle."""
     _check_gemm(zq, T, N, K, g, 4, seed=T + K)
     _check_gemm(zq, T, N, K, g, 4, seed=T + K + 1, path=2)
+
+
+@pytest.mark.parametrize("T,N,K,g", [(1, 256, 64, 4), (7, 768, 768, 48), (300, 1000, 512, 3),
+                                     (1100, 640, 2048, 5), (2048, 256, 3072, 4),
+                                     (513, 2304, 800, 48), (1024, 1024, 1024, 16)])
+@pytest.mark.parametrize("pair", [1, 2])
+def test_gemm_w4_widened_then_int8(zq, T, N, K, g, pair):
+    """INT4 weights widened once into the library workspace (an HBM-bound
+    pass), then the INT8 GEMM on the widened codes, single CTAs or CTA pairs;
+    automatic from 1024 tokens, forced here at every size."""
+    _check_gemm(zq, T, N, K, g, 4, seed=T + N + pair, path=4, pair=pair)
+
+
+def test_gemm_w4_widened_after_a_larger_call_and_reserve(zq):
+    """The workspace holds the widened codes of the largest call so far; a
+    smaller call after it, and calls after an explicit reservation, still
+    match the oracle."""
+    zq.workspace_reserve(8 << 20)
+    _check_gemm(zq, 1024, 2048, 2048, 8, 4, seed=91)
+    _check_gemm(zq, 1030, 520, 1056, 8, 4, seed=92)
+    _check_gemm(zq, 8, 1024, 2048, 8, 8, seed=93, path=2, split_k=4)
+    _check_gemm(zq, 1024, 2048, 2048, 8, 4, seed=94)
 
 
 @pytest.mark.parametrize("bits", [8, 4])

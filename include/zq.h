@@ -166,9 +166,9 @@ zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,
  * get INT4": FFN weights in INT4).  Wq4 is uint8 [N][K/2] in the layout of
  * zq_quantize_weights_groupwise(bits=4).  The nibbles are widened to int8
  * codes before the tensor-core MMAs read them:
- *   - T >= 1024 (prefill): once per call, by an HBM-bound pass into the
+ *   - T >= 512 (prefill): once per call, by an HBM-bound pass into the
  *     library workspace (N*K bytes), which the INT8 GEMM then reads;
- *   - 128 < T < 1024: in shared memory, inside each token-row tile;
+ *   - 128 < T < 512: in shared memory, inside each token-row tile;
  *   - 4 < T <= 128: in tensor memory (the MMA's A operand), inside each
  *     weight-row tile;
  *   - T <= 4: in registers, on the CUDA-core matrix-vector path.
@@ -266,7 +266,7 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  *                          INT4 weights and at T <= 2 with INT8 ones;
  *                      4 = INT4 weights widened into the workspace, then
  *                          the INT8 GEMM (zq_gemm_w4a8 only, else
- *                          ZQ_ERR_UNSUPPORTED); automatic at T >= 1024.
+ *                          ZQ_ERR_UNSUPPORTED); automatic at T >= 512.
  *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256);
  *                      the FP16-activation GEMMs accept 128 or 256 (other
  *                      values: ZQ_ERR_UNSUPPORTED) and ignore the path.
@@ -292,7 +292,7 @@ int zq_get_option(int key);
  * already), so that later GEMM calls of up to that need allocate nothing.
  * The need of a call: 4 * splits * T * N bytes for a split-K weight-streaming
  * plan, plus N * K bytes (rounded up to 256) when zq_gemm_w4a8 widens its
- * codes (T >= 1024, or ZQ_OPT_GEMM_PATH = 4).  Synchronous; call it
+ * codes (T >= 512, or ZQ_OPT_GEMM_PATH = 4).  Synchronous; call it
  * outside stream capture.  Returns ZQ_ERR_CUDA if the allocation fails.
  */
 zq_status zq_workspace_reserve(unsigned long long bytes);

@@ -177,6 +177,9 @@ struct GemmParams {
   // unit order: 0 = M tiles fastest (consecutive units, which run at the
   // same time, share their N-side operand tile), 1 = N tiles fastest
   int n_fastest;
+  // INT4 weight streaming: map_act is a 3-D map that fetches the KPS
+  // activation K slices of a stage in one box (K a multiple of KPS * 128)
+  int act3d;
 };
 
 struct Unit {
@@ -306,7 +309,19 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   if constexpr (C::PAIR) cluster_sync_all();  // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  // Set-up above touches no global memory; everything below may read what
+  // Weight streaming: ask L2 for this CTA's first weight boxes before
+  // waiting for the previous kernel of the stream (a fused LayerNorm +
+  // quantization), so that the HBM stream starts while it runs.  Only L2 is
+  // touched, which every kernel's writes reach coherently, so a weight
+  // written by that kernel cannot be read stale.
+  if (C::WROWS && threadIdx.x == 0 && static_cast<int>(unit0) < p.num_units) {
+    const Unit t = decode_unit(unit0, p);
+    const int kpb = C::W4 ? C::KPS : 1;  // K slices per weight box
+    const int kb_end = min(t.kb1, t.kb0 + 12 * kpb);
+    for (int kb = t.kb0; kb < kb_end; kb += kpb)
+      tma_prefetch_l2_2d(&map_w, C::W4 ? kb * (BK / 2) : kb * BK, t.m * BM);
+  }
+  // Set-up above writes no global memory; everything below may read what
   // the previous kernel of the stream wrote, or overwrite what it reads.
   grid_dependency_wait();
   grid_launch_dependents();
@@ -348,10 +363,15 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           // tiles (a slice past K reads the TMA's zero fill: it adds nothing)
           tma_load_2d(sP + stage * C::P_BYTES, &map_w, &pfull_bar[stage], kb * (BK / 2), t.m * BM,
                       pol_w);
+          if (p.act3d) {
+            tma_load_3d(sB + stage * C::B_BYTES, &map_act, &pfull_bar[stage], 0, t.n * BN, kb,
+                        pol_act);
+          } else {
 #pragma unroll
-          for (int h = 0; h < C::KPS; ++h)
-            tma_load_2d(sB + stage * C::B_BYTES + h * C::B_SLICE, &map_act, &pfull_bar[stage],
-                        (kb + h) * BK, t.n * BN, pol_act);
+            for (int h = 0; h < C::KPS; ++h)
+              tma_load_2d(sB + stage * C::B_BYTES + h * C::B_SLICE, &map_act, &pfull_bar[stage],
+                          (kb + h) * BK, t.n * BN, pol_act);
+          }
           ++fills[stage];
           if (++stage == C::PSTAGES) {
             stage = 0;
@@ -1038,7 +1058,7 @@ int gemv_max_tokens(bool w4) { return w4 ? kGemvMaxTokens : 2; }
 // The automatic choice of weight rows on the MMA M side (above the
 // matrix-vector range).  INT8 weights: up to 256 tokens (weight streaming).
 // INT4 weights: up to 128 tokens, where the widened weights live in tensor
-// memory next to the accumulators; from 1024 tokens the widening pass and
+// memory next to the accumulators; from 512 tokens the widening pass and
 // the INT8 GEMM take over (kWidenMinTokens), and in between the token-row
 // tiles widen the weights through shared memory.
 bool use_weight_rows(int T, int K, bool w4) {
@@ -1230,9 +1250,11 @@ struct Choice {
 };
 
 // INT4 weights at prefill-sized token counts take the widening pass and the
-// INT8 GEMM (widen_w4_kernel): from 1024 tokens up, the pass costs well
-// under a tenth of the GEMM.
-constexpr int kWidenMinTokens = 1024;
+// INT8 GEMM (widen_w4_kernel).  Measured on B200 (GPT-NeoX FFN1/FFN2): at 512
+// tokens 107/117 us against 121/135 us for the token-row tiles that widen
+// through shared memory; at 256 tokens the tiles are ahead (79 against
+// 123 us), the pass then being a third of the time.
+constexpr int kWidenMinTokens = 512;
 
 zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
   const int sms = num_sms();
@@ -1331,9 +1353,17 @@ zq_status launch_choice(bool w4, const Choice& ch, const int8_t* Xq, const float
   const int act_rows = plan.wrows ? plan.bn : BM;
   const int w_rows = plan.wrows ? BM : (plan.pair ? plan.bn / 2 : plan.bn);
   CUtensorMap ma, mw, my;
-  if (!encode_tma_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, T, K, BK, act_rows,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
+  // INT4 weight streaming (deep ring, several K slices per stage): when K is
+  // a whole number of stages, one 3-D box brings all of a stage's activation
+  // slices (one TMA copy instead of plan.kps)
+  gp.act3d = w4 && plan.wrows && plan.kps > 1 && K % (plan.kps * BK) == 0;
+  if (gp.act3d) {
+    if (!encode_tma_3d_slices(&ma, Xq, K, T, BK, act_rows, plan.kps, CU_TENSOR_MAP_SWIZZLE_128B))
+      return ZQ_ERR_CUDA;
+  } else if (!encode_tma_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, K, T, K, BK, act_rows,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) {
     return ZQ_ERR_CUDA;
+  }
   if (w4) {
     // one box per stage: plan.kps K slices of 64 packed bytes per row; with
     // the TMEM operand ring (weight rows, BN <= 128) each thread reads a

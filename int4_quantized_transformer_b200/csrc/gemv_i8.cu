@@ -67,9 +67,6 @@ __global__ void __launch_bounds__(kGemvThreads)
   constexpr int kUnroll = GemvShape<TT>::UNROLL;
   constexpr int kWarps = kGemvThreads / 32;
   __shared__ int red[kWarps][kRows * TT];
-  // Xq and s_tok may be written by the previous kernel of the stream
-  grid_dependency_wait();
-  grid_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int rg = warp / KS, ks = warp % KS;  // row group, K range
@@ -78,6 +75,26 @@ __global__ void __launch_bounds__(kGemvThreads)
   const int per = (chunks + KS - 1) / KS;
   const int cbeg = ks * per, cend = min(chunks, cbeg + per);
   const size_t row_bytes = static_cast<size_t>(K) * BITS / 8;
+  // The CTA's first block of weight rows (contiguous) goes to L2 before the
+  // wait for the previous kernel, so the HBM stream starts while it runs
+  // (only L2 is touched: the weights cannot be read stale).
+  if (threadIdx.x == 0) {
+    const int r0 = blockIdx.x * groups * kRows;
+    const int nr = min(groups * kRows, N - r0);
+    if (nr > 0) {
+      const char* base = reinterpret_cast<const char*>(W) + static_cast<size_t>(r0) * row_bytes;
+      size_t left = static_cast<size_t>(nr) * row_bytes;
+      while (left > 0) {  // row_bytes is a multiple of 16
+        const uint32_t n = static_cast<uint32_t>(left < (1u << 20) ? left : (1u << 20));
+        bulk_prefetch_l2(base, n);
+        base += n;
+        left -= n;
+      }
+    }
+  }
+  // Xq and s_tok may be written by the previous kernel of the stream
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   // every warp of the CTA runs the same number of iterations (the bound
   // depends only on blockIdx), so the __syncthreads below are uniform

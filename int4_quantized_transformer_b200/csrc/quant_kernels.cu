@@ -18,8 +18,6 @@
 // with respect to the op-by-op definition in include/zq.h.
 #include <cuda_fp16.h>
 
-#include <atomic>
-
 #include "zq_internal.h"
 #include "zq_ptx.cuh"
 
@@ -146,11 +144,9 @@ __device__ __forceinline__ float row_tree_sum(float (&cs)[VPT], float* red, int 
   return v[0];
 }
 
-// Packed and mixed-precision fp32 arithmetic of sm_100 (PTX ISA 8.6): two
-// independent IEEE round-to-nearest operations per instruction (f32x2), and
-// an add or subtract whose first operand is fp16 (converted exactly, then
-// one rounding).  They give the same bits as the scalar operations, with
-// fewer instructions per element.
+// Packed fp32 arithmetic of sm_100 (PTX ISA 8.6): two independent IEEE
+// round-to-nearest operations per instruction (f32x2).  They give the same
+// bits as the scalar operations, with fewer instructions per element.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -174,20 +170,6 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
-// f32(h) + c and f32(h) - c, one rounding each
-__device__ __forceinline__ float add_h(uint16_t h, float c) {
-  float r;
-  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(r) : "h"(h), "f"(c));
-  return r;
-}
-__device__ __forceinline__ float sub_h(uint16_t h, float c) {
-  float r;
-  asm("sub.rn.f32.f16 %0, %1, %2;" : "=f"(r) : "h"(h), "f"(c));
-  return r;
-}
-__device__ __forceinline__ void halves(uint32_t w, uint16_t& lo, uint16_t& hi) {
-  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
-}
 // running max of |.| over packed fp16 pairs (the sign of the result is
 // meaningless; its magnitude is max(|a|, |b|) per half)
 __device__ __forceinline__ uint32_t hmax_abs2(uint32_t a, uint32_t b) {
@@ -195,61 +177,36 @@ __device__ __forceinline__ uint32_t hmax_abs2(uint32_t a, uint32_t b) {
   asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
+__device__ __forceinline__ float habs_max(uint32_t m2) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&m2));
+  return fmaxf(fabsf(f.x), fabsf(f.y));
+}
 
-// LayerNorm gamma/beta are kept as fp32 in shared memory (converted once per
-// CTA) when both fit in this many bytes; longer rows convert per row.
-constexpr int kGammaBetaSmemMax = 64 * 1024;
+// ------------------------------------------------- token quantization only
 
-// W warps per row, VPT 16-byte vectors (8 halves) per thread.  Blocks hold
-// RPB = max(1, 8/W) rows; every thread runs the same number of row
-// iterations so block-wide barriers stay uniform.  The loads of a thread's
-// next row are issued before the current row is reduced, so their latency
-// overlaps its arithmetic.
+// One row per group of W warps, VPT 16-byte vectors (8 halves) per thread:
+// the quant-only form of zq_ln_quant, zq_bias_act_quant (act >= 0: the
+// bias-add or GeLU producer fused in front) and zq_static_quant
+// (static_amax >= 0).  Blocks hold RPB = max(1, 8/W) rows; every thread
+// runs the same number of row iterations so block-wide barriers stay
+// uniform.  The loads of a thread's next row are issued before the current
+// row is reduced, so their latency overlaps its arithmetic.
 template <int W, int VPT>
-__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
-    ln_quant_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
-                    const __half* __restrict__ beta, const __half* __restrict__ act_bias,
-                    int act, float static_amax, int T, int K, float eps,
-                    int8_t* __restrict__ Xq, float* __restrict__ s_tok,
-                    __half* __restrict__ Y_ln) {
+__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 32) : 8) / 2)
+    quant_rows_kernel(const __half* __restrict__ X, const __half* __restrict__ act_bias, int act,
+                      float static_amax, int T, int K, int8_t* __restrict__ Xq,
+                      float* __restrict__ s_tok, __half* __restrict__ Y_out) {
   constexpr int RT = 32 * W;                // threads per row
   constexpr int RPB = W >= 8 ? 1 : 8 / W;   // rows per block
-  constexpr int NBLK = W * (VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4));
-  __shared__ float red1[RPB][NBLK];  // block sums of x (W > 1)
-  __shared__ float red2[RPB][NBLK];  // block sums of (x - mean)^2 (W > 1)
   __shared__ float red_m[RPB][W];
-  extern __shared__ float4 gb_smem[];  // fp32 gamma [K], then beta [K] (when they fit)
 
   const int slot = threadIdx.x / RT;
   const int j = threadIdx.x % RT;
   const int warp_in_row = j / 32;
   const int lane = threadIdx.x & 31;
   const int nvec = K / 8;
-  const bool ln = gamma != nullptr;
-  const bool gb_smem_ok = ln && 8 * K <= kGammaBetaSmemMax;
-  const float* g_s = reinterpret_cast<const float*>(gb_smem);
-  const float* b_s = g_s + K;
   grid_dependency_wait();
   grid_launch_dependents();
-  if (gb_smem_ok) {
-    float* gs = reinterpret_cast<float*>(gb_smem);
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-      const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
-      const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v) : make_uint4(0, 0, 0, 0);
-      const __half2* gh = reinterpret_cast<const __half2*>(&g4);
-      const __half2* bh = reinterpret_cast<const __half2*>(&b4);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 gf = __half22float2(gh[e]);
-        const float2 bf = __half22float2(bh[e]);
-        gs[8 * v + 2 * e] = gf.x;
-        gs[8 * v + 2 * e + 1] = gf.y;
-        gs[K + 8 * v + 2 * e] = bf.x;
-        gs[K + 8 * v + 2 * e + 1] = bf.y;
-      }
-    }
-    __syncthreads();
-  }
 
   const int rows_per_iter = gridDim.x * RPB;
   const int iters = (T + rows_per_iter - 1) / rows_per_iter;
@@ -300,133 +257,28 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
       }
     }
 
-    if (ln) {
-      // mean: each 8-element chunk summed in index order (the first element
-      // plus -0 is the element itself, exactly), then the pairwise tree
-      float cs[VPT];
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
-        float acc = -0.0f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint16_t lo, hi;
-          halves(w[e], lo, hi);
-          acc = add_h(hi, add_h(lo, acc));
-        }
-        cs[i] = acc;  // zero for chunks past the row (x4 is zero there)
-      }
-      const float mean = __fdiv_rn(row_tree_sum<W, VPT>(cs, red1[slot], lane, warp_in_row),
-                                   static_cast<float>(K));
-      // deviations x - mean (kept for the normalisation), then the biased
-      // variance: per chunk the first square, then fused multiply-adds in
-      // index order, two chunks at a time in the two halves of f32x2
-      float d[VPT][8];
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint16_t lo, hi;
-          halves(w[e], lo, hi);
-          d[i][2 * e] = sub_h(lo, mean);
-          d[i][2 * e + 1] = sub_h(hi, mean);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i + 1 < VPT; i += 2) {
-        uint64_t q = f2_pack(d[i][0], d[i + 1][0]);
-        q = f2_mul(q, q);
-#pragma unroll
-        for (int e = 1; e < 8; ++e) {
-          const uint64_t de = f2_pack(d[i][e], d[i + 1][e]);
-          q = f2_fma(de, de, q);
-        }
-        f2_unpack(q, cs[i], cs[i + 1]);
-      }
-      if (VPT % 2) {
-        float acc = __fmul_rn(d[VPT - 1][0], d[VPT - 1][0]);
-#pragma unroll
-        for (int e = 1; e < 8; ++e) acc = __fmaf_rn(d[VPT - 1][e], d[VPT - 1][e], acc);
-        cs[VPT - 1] = acc;
-      }
-#pragma unroll
-      for (int i = 0; i < VPT; ++i)
-        if (j + i * RT >= nvec) cs[i] = 0.0f;  // padding chunks are zero
-      const float var = __fdiv_rn(row_tree_sum<W, VPT>(cs, red2[slot], lane, warp_in_row),
-                                  static_cast<float>(K));
-      const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, eps)));
-      const uint64_t rstd2 = f2_pack(rstd, rstd);
-      // y = fp16(((x - mean) * rstd) * gamma + beta), each step rounded once
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        const int v = j + i * RT;
-        if (v < nvec) {
-          float g[8], b[8];
-          if (gb_smem_ok) {
-            const float4* gp = reinterpret_cast<const float4*>(g_s + 8 * v);
-            const float4* bp = reinterpret_cast<const float4*>(b_s + 8 * v);
-            const float4 g0 = gp[0], g1 = gp[1], b0 = bp[0], b1 = bp[1];
-            g[0] = g0.x; g[1] = g0.y; g[2] = g0.z; g[3] = g0.w;
-            g[4] = g1.x; g[5] = g1.y; g[6] = g1.z; g[7] = g1.w;
-            b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
-            b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
-          } else {
-            const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
-            const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v)
-                                  : make_uint4(0, 0, 0, 0);
-            const __half2* gh = reinterpret_cast<const __half2*>(&g4);
-            const __half2* bh = reinterpret_cast<const __half2*>(&b4);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 gf = __half22float2(gh[e]);
-              const float2 bf = __half22float2(bh[e]);
-              g[2 * e] = gf.x;
-              g[2 * e + 1] = gf.y;
-              b[2 * e] = bf.x;
-              b[2 * e + 1] = bf.y;
-            }
-          }
-          __half2* h = reinterpret_cast<__half2*>(&x4[i]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            uint64_t t = f2_mul(f2_pack(d[i][2 * e], d[i][2 * e + 1]), rstd2);
-            t = f2_mul(t, f2_pack(g[2 * e], g[2 * e + 1]));
-            t = f2_add(t, f2_pack(b[2 * e], b[2 * e + 1]));
-            float y0, y1;
-            f2_unpack(t, y0, y1);
-            h[e] = __floats2half2_rn(y0, y1);
-          }
-        }
-      }
-    }
-
-    // absmax of the fp16 row (padding vectors are zero)
-    uint32_t m2 = 0u;
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) m2 = hmax_abs2(m2, w[e]);
-    }
     // static quantization: one calibrated range for every token (codes may
     // then exceed the range and are clamped), no per-row reduction
     const bool is_static = static_amax >= 0.0f;  // uniform over the grid
     float amax = static_amax;
     if (!is_static) {
-      const float2 mf = __half22float2(*reinterpret_cast<const __half2*>(&m2));
-      amax = warp_max(fmaxf(fabsf(mf.x), fabsf(mf.y)));
+      uint32_t m2 = 0u;  // padding vectors are zero
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&x4[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m2 = hmax_abs2(m2, w[e]);
+      }
+      amax = warp_max(habs_max(m2));
       if (W > 1) {
         if (lane == 0) red_m[slot][warp_in_row] = amax;
         __syncthreads();
 #pragma unroll
         for (int w = 0; w < W; ++w) amax = fmaxf(amax, red_m[slot][w]);
-        __syncthreads();  // red1 / red2 / red_m are reused by the next row
+        __syncthreads();  // red_m is reused by the next row
       }
     }
     const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-    const uint64_t inv2 = f2_pack(inv, inv);
-    const uint64_t magic2 = f2_pack(12582912.0f, 12582912.0f);
     if (valid) {
       if (j == 0) s_tok[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
       int8_t* qr = Xq + static_cast<size_t>(row) * K;
@@ -439,23 +291,14 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __half22float2(h[e]);
-            if (is_static) {
-              c[2 * e] = quant_code(f.x, inv, 127.0f);
-              c[2 * e + 1] = quant_code(f.y, inv, 127.0f);
-            } else {
-              // rne(y * inv) in the low byte: the product, then + 1.5 * 2^23
-              const uint64_t t = f2_add(f2_mul(f2_pack(f.x, f.y), inv2), magic2);
-              float a, b;
-              f2_unpack(t, a, b);
-              c[2 * e] = __float_as_uint(a);
-              c[2 * e + 1] = __float_as_uint(b);
-            }
+            c[2 * e] = is_static ? quant_code(f.x, inv, 127.0f) : token_code(f.x, inv);
+            c[2 * e + 1] = is_static ? quant_code(f.y, inv, 127.0f) : token_code(f.y, inv);
           }
           uint2 out;
           out.x = pack4(c[0], c[1], c[2], c[3]);
           out.y = pack4(c[4], c[5], c[6], c[7]);
           __stcs(reinterpret_cast<uint2*>(qr) + v, out);
-          if (Y_ln) reinterpret_cast<uint4*>(Y_ln + static_cast<size_t>(row) * K)[v] = x4[i];
+          if (Y_out) reinterpret_cast<uint4*>(Y_out + static_cast<size_t>(row) * K)[v] = x4[i];
         }
       }
     }
@@ -464,68 +307,324 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
   }
 }
 
+// ---------------------------------------------------------- LN + quant
+
+// The fixed-order tree of row_tree_sum for two rows at once: the low and
+// high halves of each f32x2 value are rows A and B, and every add is the
+// same IEEE operation as in the one-row tree.
 template <int W, int VPT>
-cudaError_t launch_ln(const __half* X, const __half* g, const __half* b, const __half* ab, int act,
-                      float sa, int T, int K, float eps, int8_t* Xq, float* s, __half* Y,
-                      cudaStream_t st) {
-  constexpr int RPB = W >= 8 ? 1 : 8 / W;
-  constexpr int threads = RPB * 32 * W;
-  const size_t smem = (g && 8 * K <= kGammaBetaSmemMax) ? static_cast<size_t>(8) * K : 0;
-  // per device; several host threads may race here, and a repeated set is
-  // harmless
-  static std::atomic<bool> attr_set[64];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-    e = cudaFuncSetAttribute(ln_quant_kernel<W, VPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kGammaBetaSmemMax);
-    if (e != cudaSuccess) return e;
-    attr_set[dev].store(true, std::memory_order_release);
+__device__ __forceinline__ uint64_t row_tree_sum2(uint64_t (&cs)[VPT], uint64_t* red, int lane,
+                                                  int wrow) {
+  constexpr int VPTP = VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) cs[i] = f2_add(cs[i], __shfl_xor_sync(0xffffffffu, cs[i], o));
+  if (W == 1) {
+    uint64_t b[VPTP];
+#pragma unroll
+    for (int i = 0; i < VPTP; ++i) b[i] = i < VPT ? cs[i] : 0ull;
+#pragma unroll
+    for (int st = 1; st < VPTP; st <<= 1)
+#pragma unroll
+      for (int i = 0; i < VPTP; i += 2 * st) b[i] = f2_add(b[i], b[i + st]);
+    return b[0];
   }
+  constexpr int NB = W * VPTP;
+  constexpr int NR = NB <= 32 ? 1 : NB / 32;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < VPTP; ++i) red[wrow + W * i] = i < VPT ? cs[i] : 0ull;
+  }
+  __syncthreads();
+  uint64_t v[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) v[r] = (lane + 32 * r < NB) ? red[lane + 32 * r] : 0ull;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+    for (int r = 0; r < NR; ++r) v[r] = f2_add(v[r], __shfl_xor_sync(0xffffffffu, v[r], o));
+#pragma unroll
+  for (int st = 1; st < NR; st <<= 1)
+#pragma unroll
+    for (int r = 0; r < NR; r += 2 * st) v[r] = f2_add(v[r], v[r + st]);
+  return v[0];
+}
+
+// Fused LayerNorm + token quantization, two rows (A = 2p, B = 2p + 1) per
+// group of W warps.  Each thread holds VPT 16-byte vectors of both rows and
+// keeps every per-column value as an f32x2 pair (row A, row B), so the
+// statistics, the deviations and the quantization run two rows per
+// instruction with the one-row operation order: chunk sums in index order,
+// the fixed tree, the two-pass variance with fused multiply-adds, then
+// y = fp16(((x - mean) * rstd) * gamma + beta) with each step rounded once.
+// Blocks hold PPB = max(1, 8/W) row pairs; the next pair's loads are issued
+// before the current pair is reduced.
+template <int W, int VPT>
+__global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
+    ln_rows2_kernel(const __half* __restrict__ X, const __half* __restrict__ gamma,
+                    const __half* __restrict__ beta, int T, int K, float eps,
+                    int8_t* __restrict__ Xq, float* __restrict__ s_tok,
+                    __half* __restrict__ Y_ln) {
+  constexpr int RT = 32 * W;                // threads per row pair
+  constexpr int PPB = W >= 8 ? 1 : 8 / W;   // row pairs per block
+  constexpr int NBLK = W * (VPT <= 1 ? 1 : (VPT <= 2 ? 2 : 4));
+  __shared__ uint64_t red1[PPB][NBLK];  // block sums of x (W > 1)
+  __shared__ uint64_t red2[PPB][NBLK];  // block sums of (x - mean)^2 (W > 1)
+  __shared__ float red_m[PPB][2][W];
+
+  const int slot = threadIdx.x / RT;
+  const int j = threadIdx.x % RT;
+  const int warp_in_row = j / 32;
+  const int lane = threadIdx.x & 31;
+  const int nvec = K / 8;
+  grid_dependency_wait();
+  grid_launch_dependents();
+
+  const int pairs = (T + 1) / 2;
+  const int pairs_per_iter = gridDim.x * PPB;
+  const int iters = (pairs + pairs_per_iter - 1) / pairs_per_iter;
+  auto load_pair = [&](uint4 (&a)[VPT], uint4 (&b)[VPT], int p) {
+    const __half* xa = X + static_cast<size_t>(2 * p) * K;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = j + i * RT;
+      a[i] = make_uint4(0, 0, 0, 0);
+      b[i] = make_uint4(0, 0, 0, 0);
+      if (v < nvec) {
+        if (2 * p < T) a[i] = __ldcs(reinterpret_cast<const uint4*>(xa) + v);
+        if (2 * p + 1 < T) b[i] = __ldcs(reinterpret_cast<const uint4*>(xa + K) + v);
+      }
+    }
+  };
+  uint4 xa[VPT], xb[VPT];
+  load_pair(xa, xb, blockIdx.x * PPB + slot);
+  for (int it = 0; it < iters; ++it) {
+    const int p = (it * gridDim.x + blockIdx.x) * PPB + slot;
+    uint4 na[VPT], nb[VPT];
+    if (it + 1 < iters) load_pair(na, nb, ((it + 1) * gridDim.x + blockIdx.x) * PPB + slot);
+
+    // x as (row A, row B) pairs; chunk sums in index order
+    uint64_t P[VPT][8];
+    uint64_t cs[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const __half* ha = reinterpret_cast<const __half*>(&xa[i]);
+      const __half* hb = reinterpret_cast<const __half*>(&xb[i]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) P[i][e] = f2_pack(__half2float(ha[e]), __half2float(hb[e]));
+      uint64_t acc = f2_add(P[i][0], P[i][1]);
+#pragma unroll
+      for (int e = 2; e < 8; ++e) acc = f2_add(acc, P[i][e]);
+      cs[i] = acc;  // zero for chunks past the row (the vectors are zero there)
+    }
+    float sa, sb;
+    f2_unpack(row_tree_sum2<W, VPT>(cs, red1[slot], lane, warp_in_row), sa, sb);
+    const float mean_a = __fdiv_rn(sa, static_cast<float>(K));
+    const float mean_b = __fdiv_rn(sb, static_cast<float>(K));
+    // deviations x - mean (as x + (-mean), the same IEEE operation), then the
+    // biased variance: per chunk the first square, then fused multiply-adds
+    const uint64_t negm = f2_pack(-mean_a, -mean_b);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) P[i][e] = f2_add(P[i][e], negm);
+      uint64_t q = f2_mul(P[i][0], P[i][0]);
+#pragma unroll
+      for (int e = 1; e < 8; ++e) q = f2_fma(P[i][e], P[i][e], q);
+      cs[i] = (j + i * RT < nvec) ? q : 0ull;  // padding chunks are zero
+    }
+    f2_unpack(row_tree_sum2<W, VPT>(cs, red2[slot], lane, warp_in_row), sa, sb);
+    const float var_a = __fdiv_rn(sa, static_cast<float>(K));
+    const float var_b = __fdiv_rn(sb, static_cast<float>(K));
+    const uint64_t rstd2 = f2_pack(__fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var_a, eps))),
+                                   __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var_b, eps))));
+    // y = fp16(((x - mean) * rstd) * gamma + beta): the first product for
+    // both rows at once, gamma and beta (shared by the rows) one row at a time
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = j + i * RT;
+      if (v < nvec) {
+        const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(gamma) + v);
+        const uint4 b4 = beta ? __ldg(reinterpret_cast<const uint4*>(beta) + v)
+                              : make_uint4(0, 0, 0, 0);
+        const __half2* gh = reinterpret_cast<const __half2*>(&g4);
+        const __half2* bh = reinterpret_cast<const __half2*>(&b4);
+        __half2* ya = reinterpret_cast<__half2*>(&xa[i]);
+        __half2* yb = reinterpret_cast<__half2*>(&xb[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 gf = __half22float2(gh[e]);
+          const float2 bf = __half22float2(bh[e]);
+          float a0, b0, a1, b1;
+          f2_unpack(f2_mul(P[i][2 * e], rstd2), a0, b0);
+          f2_unpack(f2_mul(P[i][2 * e + 1], rstd2), a1, b1);
+          ya[e] = __floats2half2_rn(__fadd_rn(__fmul_rn(a0, gf.x), bf.x),
+                                    __fadd_rn(__fmul_rn(a1, gf.y), bf.y));
+          yb[e] = __floats2half2_rn(__fadd_rn(__fmul_rn(b0, gf.x), bf.x),
+                                    __fadd_rn(__fmul_rn(b1, gf.y), bf.y));
+        }
+      } else {
+        xa[i] = make_uint4(0, 0, 0, 0);
+        xb[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    // absmax of both fp16 rows
+    uint32_t ma = 0u, mb = 0u;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const uint32_t* wa = reinterpret_cast<const uint32_t*>(&xa[i]);
+      const uint32_t* wb = reinterpret_cast<const uint32_t*>(&xb[i]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ma = hmax_abs2(ma, wa[e]);
+        mb = hmax_abs2(mb, wb[e]);
+      }
+    }
+    float amax_a = warp_max(habs_max(ma));
+    float amax_b = warp_max(habs_max(mb));
+    if (W > 1) {
+      if (lane == 0) {
+        red_m[slot][0][warp_in_row] = amax_a;
+        red_m[slot][1][warp_in_row] = amax_b;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        amax_a = fmaxf(amax_a, red_m[slot][0][w]);
+        amax_b = fmaxf(amax_b, red_m[slot][1][w]);
+      }
+      __syncthreads();  // red1 / red2 / red_m are reused by the next pair
+    }
+    const float inv_a = amax_a > 0.0f ? __fdiv_rn(127.0f, amax_a) : 0.0f;
+    const float inv_b = amax_b > 0.0f ? __fdiv_rn(127.0f, amax_b) : 0.0f;
+    const int ra = 2 * p, rb = 2 * p + 1;
+    if (j == 0) {
+      if (ra < T) s_tok[ra] = amax_a > 0.0f ? __fdiv_rn(amax_a, 127.0f) : 0.0f;
+      if (rb < T) s_tok[rb] = amax_b > 0.0f ? __fdiv_rn(amax_b, 127.0f) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int v = j + i * RT;
+      if (v < nvec) {
+        const __half2* ya = reinterpret_cast<const __half2*>(&xa[i]);
+        const __half2* yb = reinterpret_cast<const __half2*>(&xb[i]);
+        uint32_t ca[8], cb[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fa = __half22float2(ya[e]);
+          const float2 fb = __half22float2(yb[e]);
+          ca[2 * e] = token_code(fa.x, inv_a);
+          ca[2 * e + 1] = token_code(fa.y, inv_a);
+          cb[2 * e] = token_code(fb.x, inv_b);
+          cb[2 * e + 1] = token_code(fb.y, inv_b);
+        }
+        if (ra < T) {
+          __stcs(reinterpret_cast<uint2*>(Xq + static_cast<size_t>(ra) * K) + v,
+                 make_uint2(pack4(ca[0], ca[1], ca[2], ca[3]), pack4(ca[4], ca[5], ca[6], ca[7])));
+          if (Y_ln) reinterpret_cast<uint4*>(Y_ln + static_cast<size_t>(ra) * K)[v] = xa[i];
+        }
+        if (rb < T) {
+          __stcs(reinterpret_cast<uint2*>(Xq + static_cast<size_t>(rb) * K) + v,
+                 make_uint2(pack4(cb[0], cb[1], cb[2], cb[3]), pack4(cb[4], cb[5], cb[6], cb[7])));
+          if (Y_ln) reinterpret_cast<uint4*>(Y_ln + static_cast<size_t>(rb) * K)[v] = xb[i];
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      xa[i] = na[i];
+      xb[i] = nb[i];
+    }
+  }
+}
+
+// Launches on as many CTAs as are resident at once, or fewer when there are
+// fewer row groups (the row loop is grid-strided).
+template <class Kern, class... Args>
+cudaError_t launch_resident(Kern kernel, int threads, int groups, cudaStream_t st, Args... args) {
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ln_quant_kernel<W, VPT>, threads,
-                                                    smem);
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  int need = (T + RPB - 1) / RPB;
   int grid = num_sms() * per_sm;
-  if (grid > need) grid = need;
-  e = launch_pdl(ln_quant_kernel<W, VPT>, dim3(grid), dim3(threads), smem, st, X, g, b, ab, act,
-                 sa, T, K, eps, Xq, s, Y);
+  if (grid > groups) grid = groups;
+  if (grid < 1) grid = 1;
+  e = launch_pdl(kernel, dim3(grid), dim3(threads), 0, st, args...);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
+template <int W, int VPT>
+cudaError_t launch_quant_rows(const __half* X, const __half* ab, int act, float sa, int T, int K,
+                              int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
+  constexpr int RPB = W >= 8 ? 1 : 8 / W;
+  return launch_resident(quant_rows_kernel<W, VPT>, RPB * 32 * W, (T + RPB - 1) / RPB, st, X, ab,
+                         act, sa, T, K, Xq, s, Y);
+}
+
+template <int W, int VPT>
+cudaError_t launch_ln_rows2(const __half* X, const __half* g, const __half* b, int T, int K,
+                            float eps, int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
+  constexpr int PPB = W >= 8 ? 1 : 8 / W;
+  const int pairs = (T + 1) / 2;
+  return launch_resident(ln_rows2_kernel<W, VPT>, PPB * 32 * W, (pairs + PPB - 1) / PPB, st, X, g,
+                         b, T, K, eps, Xq, s, Y);
+}
+
+#define ZQ_VPT_SWITCH(FN, W, vpt, ...)                  \
+  switch (vpt) {                                        \
+    case 1: return FN<W, 1>(__VA_ARGS__);               \
+    case 2: return FN<W, 2>(__VA_ARGS__);               \
+    case 3: return FN<W, 3>(__VA_ARGS__);               \
+    default: return FN<W, 4>(__VA_ARGS__);              \
+  }
+
 template <int W>
-cudaError_t launch_ln_w(int vpt, const __half* X, const __half* g, const __half* b,
-                        const __half* ab, int act, float sa, int T, int K, float eps, int8_t* Xq,
-                        float* s, __half* Y, cudaStream_t st) {
+cudaError_t launch_quant_w(int vpt, const __half* X, const __half* ab, int act, float sa, int T,
+                           int K, int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
+  ZQ_VPT_SWITCH(launch_quant_rows, W, vpt, X, ab, act, sa, T, K, Xq, s, Y, st)
+}
+
+template <int W>
+cudaError_t launch_ln_w(int vpt, const __half* X, const __half* g, const __half* b, int T, int K,
+                        float eps, int8_t* Xq, float* s, __half* Y, cudaStream_t st) {
   switch (vpt) {
-    case 1: return launch_ln<W, 1>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
-    case 2: return launch_ln<W, 2>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
-    case 3: return launch_ln<W, 3>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
-    default: return launch_ln<W, 4>(X, g, b, ab, act, sa, T, K, eps, Xq, s, Y, st);
+    case 1: return launch_ln_rows2<W, 1>(X, g, b, T, K, eps, Xq, s, Y, st);
+    case 2: return launch_ln_rows2<W, 2>(X, g, b, T, K, eps, Xq, s, Y, st);
+    default: return launch_ln_rows2<W, 3>(X, g, b, T, K, eps, Xq, s, Y, st);
   }
 }
 
-// Warps per row so that each thread keeps at most 4 vectors of 8 halves;
-// act < 0 selects the LayerNorm (gamma non-NULL) or quant-only form;
-// sa >= 0 is a static range (one scale for every token).
+// Warps per row so that each thread keeps at most 4 vectors of 8 halves
+// (3 for the two-row LayerNorm kernel, which holds both rows); act < 0
+// selects the LayerNorm (gamma non-NULL) or quant-only form; sa >= 0 is a
+// static range (one scale for every token).
 cudaError_t launch_row_quant(const __half* xg, const __half* gg, const __half* bg,
                              const __half* ab, int act, float sa, int T, int K, float eps,
                              int8_t* Xq, float* s_tok, __half* yg, cudaStream_t st) {
   const int nvec = K / 8;
+  const int vmax = gg ? 3 : 4;
   int W = 1;
-  while (W < 32 && 32 * W * 4 < nvec) W *= 2;
+  while (W < 32 && 32 * W * vmax < nvec) W *= 2;
   const int vpt = (nvec + 32 * W - 1) / (32 * W);
+  if (gg) {
+    switch (W) {
+      case 1: return launch_ln_w<1>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
+      case 2: return launch_ln_w<2>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
+      case 4: return launch_ln_w<4>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
+      case 8: return launch_ln_w<8>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
+      case 16: return launch_ln_w<16>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
+      default: return launch_ln_w<32>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
+    }
+  }
   switch (W) {
-    case 1: return launch_ln_w<1>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
-    case 2: return launch_ln_w<2>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
-    case 4: return launch_ln_w<4>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
-    case 8: return launch_ln_w<8>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
-    case 16: return launch_ln_w<16>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
-    default: return launch_ln_w<32>(vpt, xg, gg, bg, ab, act, sa, T, K, eps, Xq, s_tok, yg, st);
+    case 1: return launch_quant_w<1>(vpt, xg, ab, act, sa, T, K, Xq, s_tok, yg, st);
+    case 2: return launch_quant_w<2>(vpt, xg, ab, act, sa, T, K, Xq, s_tok, yg, st);
+    case 4: return launch_quant_w<4>(vpt, xg, ab, act, sa, T, K, Xq, s_tok, yg, st);
+    case 8: return launch_quant_w<8>(vpt, xg, ab, act, sa, T, K, Xq, s_tok, yg, st);
+    case 16: return launch_quant_w<16>(vpt, xg, ab, act, sa, T, K, Xq, s_tok, yg, st);
+    default: return launch_quant_w<32>(vpt, xg, ab, act, sa, T, K, Xq, s_tok, yg, st);
   }
 }
 

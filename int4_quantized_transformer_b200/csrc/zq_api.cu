@@ -88,6 +88,32 @@ bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tma_3d_slices(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                          uint32_t slice, uint32_t box_outer, uint32_t box_slices,
+                          CUtensorMapSwizzle swizzle) {
+  if (slice == 0 || inner % slice != 0) return false;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  cuuint64_t dims[3] = {slice, outer, inner / slice};
+  cuuint64_t strides[2] = {inner, slice};  // bytes: next row, next slice
+  cuuint32_t box[3] = {slice, box_outer, box_slices};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // A barrier nobody arrives at: the wait must give up by itself.
 __global__ void debug_wait_timeout_kernel(int* status) {
   __shared__ __align__(8) uint64_t bar;

@@ -42,6 +42,14 @@ bool encode_tma_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base
                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
                    uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
+// A 3-D tiled map over row-major [outer][inner] bytes viewed as
+// [inner / slice][outer][slice]: one box fetches `box_slices` consecutive
+// slices of `box_outer` rows (slice-major in shared memory).  `inner` must
+// be a multiple of `slice`.
+bool encode_tma_3d_slices(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                          uint32_t slice, uint32_t box_outer, uint32_t box_slices,
+                          CUtensorMapSwizzle swizzle);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Launches a kernel on `st` with programmatic stream serialization, so that

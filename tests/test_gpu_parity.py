@@ -186,10 +186,11 @@ def test_gemm_auto(zq, bits, T, N, K, g):
 
 
 @pytest.mark.parametrize("T,N,K,g", [(1100, 640, 2048, 5), (130, 512, 2048, 8), (128, 384, 4096, 3),
-                                     (2048, 256, 3072, 4), (1024, 1024, 1024, 16)])
+                                     (2048, 256, 3072, 4), (1024, 1024, 1024, 16),
+                                     (511, 768, 1024, 6), (512, 768, 1024, 6)])
 def test_gemm_w4_tiling_choices(zq, T, N, K, g):
     """INT4 weights choose weight-row tiles (widened weights in TMEM) up to
-    T = 128, token-row tiles up to 1024 tokens and the widening pass with the
+    T = 128, token-row tiles below 512 tokens and the widening pass with the
     INT8 GEMM from there; both sides of each boundary, and the forced
     weight-row alternative, match the oracle."""
     _check_gemm(zq, T, N, K, g, 4, seed=T + K)
@@ -203,7 +204,7 @@ def test_gemm_w4_tiling_choices(zq, T, N, K, g):
 def test_gemm_w4_widened_then_int8(zq, T, N, K, g, pair):
     """INT4 weights widened once into the library workspace (an HBM-bound
     pass), then the INT8 GEMM on the widened codes, single CTAs or CTA pairs;
-    automatic from 1024 tokens, forced here at every size."""
+    automatic from 512 tokens, forced here at every size."""
     _check_gemm(zq, T, N, K, g, 4, seed=T + N + pair, path=4, pair=pair)
 
 

@@ -173,7 +173,8 @@ struct GemmParams {
   int32_t* ws;     // split-K partial sums [splits][T][N]
   int* status;
   int T, N, K, g;
-  int m_tiles, n_tiles, k_blocks, splits, kb_per_split, num_units;
+  int m_tiles, n_tiles, k_blocks, splits, num_units;
+  int kps;  // K slices per pipeline stage (Cfg::KPS of the launched kernel)
   // unit order: 0 = M tiles fastest (consecutive units, which run at the
   // same time, share their N-side operand tile), 1 = N tiles fastest
   int n_fastest;
@@ -182,8 +183,13 @@ struct GemmParams {
   int act3d;
 };
 
+// A work unit: one output tile (m, n) and the K slices kb0, kb0 + kstep, ...
+// below kb1.  With K split across SMs (weight-row tiling), split s of S
+// takes the stages s, s + S, s + 2S, ... (stages of kps slices): at any
+// moment the S CTAs of one weight tile read adjacent pieces of its rows,
+// which the DRAM serves as longer contiguous runs than S separate ranges.
 struct Unit {
-  int m, n, kb0, kb1;
+  int m, n, kb0, kb1, kstep, split;
 };
 
 __device__ __forceinline__ Unit decode_unit(int u, const GemmParams& p) {
@@ -197,8 +203,10 @@ __device__ __forceinline__ Unit decode_unit(int u, const GemmParams& p) {
     r.m = rest % p.m_tiles;
     r.n = rest / p.m_tiles;
   }
-  r.kb0 = split * p.kb_per_split;
-  r.kb1 = min(p.k_blocks, r.kb0 + p.kb_per_split);
+  r.split = split;
+  r.kb0 = split * p.kps;
+  r.kb1 = p.k_blocks;
+  r.kstep = p.splits * p.kps;
   return r;
 }
 
@@ -316,9 +324,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   // written by that kernel cannot be read stale.
   if (C::WROWS && threadIdx.x == 0 && static_cast<int>(unit0) < p.num_units) {
     const Unit t = decode_unit(unit0, p);
-    const int kpb = C::W4 ? C::KPS : 1;  // K slices per weight box
-    const int kb_end = min(t.kb1, t.kb0 + 12 * kpb);
-    for (int kb = t.kb0; kb < kb_end; kb += kpb)
+    for (int i = 0, kb = t.kb0; i < 12 && kb < t.kb1; ++i, kb += t.kstep)  // one box per stage
       tma_prefetch_l2_2d(&map_w, C::W4 ? kb * (BK / 2) : kb * BK, t.m * BM);
   }
   // Set-up above writes no global memory; everything below may read what
@@ -346,7 +352,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ok = true;
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
-        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
+        for (int kb = t.kb0; kb < t.kb1; kb += t.kstep) {
           if (NP > 1 && (seq++ % NP) != pid) {
             if (++stage == C::PSTAGES) {
               stage = 0;
@@ -399,7 +405,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         const Unit t = decode_unit(u, p);
         const int act_row = C::WROWS ? t.n * BN : t.m * C::TILE_M + static_cast<int>(crank) * BM;
         const int w_row = C::WROWS ? t.m * BM : t.n * BN + static_cast<int>(crank) * C::W_ROWS;
-        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
+        for (int kb = t.kb0; kb < t.kb1; kb += t.kstep) {
           if (NP > 1 && (seq++ % NP) != pid) {
             if (++stage == STAGES) {
               stage = 0;
@@ -478,7 +484,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
         if (!mbar_wait(&tempty_bar[buf], tphase ^ 1, abort_flag, p.status, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * C::BUF_COLS);
-        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
+        for (int kb = t.kb0; kb < t.kb1; kb += t.kstep) {
           uint64_t* rb = C::W4 ? &ready_bar[stage] : &full_bar[stage];
           if (!mbar_wait(rb, phase, abort_flag, p.status, 3)) {
             ok = false;
@@ -655,7 +661,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
                 const int a = static_cast<int>(acc[j]);
                 const size_t idx = static_cast<size_t>(tok) * p.N + o;
                 if (split) {
-                  p.ws[static_cast<size_t>(t.kb0 / p.kb_per_split) * p.T * p.N + idx] = a;
+                  p.ws[static_cast<size_t>(t.split) * p.T * p.N + idx] = a;
                 } else {
                   float v = __fmul_rn(__int2float_rn(a), colv[c0 + j]);
                   v = __fadd_rn(__fmul_rn(v, rscale), rbias);
@@ -810,7 +816,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       bool ok = true;
       for (int u = unit0; ok && u < p.num_units; u += ustep) {
         const Unit t = decode_unit(u, p);
-        for (int kb = t.kb0; kb < t.kb1; kb += C::KPS) {
+        for (int kb = t.kb0; kb < t.kb1; kb += t.kstep) {
           if constexpr (C::DEEP) {
             // the packed slice has landed, and the MMA has released the slot
             // of the shallow ring that the unpacked weights go to
@@ -1338,7 +1344,7 @@ zq_status launch_choice(bool w4, const Choice& ch, const int8_t* Xq, const float
   gp.n_tiles = plan.n_tiles;
   gp.k_blocks = plan.k_blocks;
   gp.splits = plan.splits;
-  gp.kb_per_split = plan.kb_per_split;
+  gp.kps = plan.kps;
   gp.num_units = plan.units;
   // Weight rows with several token tiles: when the weights are the larger
   // operand, let the CTAs running at the same time share a weight tile (each

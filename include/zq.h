@@ -196,9 +196,13 @@ zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
  *   acc_dbg     fp32 [T][N] or NULL: also store acc (for checking).
  * Runs on tcgen05 tensor cores (kind::f16), except for T <= 4: a
  * memory-bound matrix-vector product on CUDA cores (exact products, fp32
- * fma sums).  ZQ_OPT_GEMM_PATH = 3 forces that path (T <= 4), 1 or 2 the
- * tensor cores; ZQ_OPT_CTA_PAIR = 2 forces 256-row units shared by a CTA
- * pair (measured slower, never chosen automatically).
+ * fma sums).  From T = 1024 the codes are first widened to fp16 integers in
+ * the library workspace (2*N*K bytes, an HBM-bound pass) and the GEMM reads
+ * them by TMA, on single CTAs or CTA pairs; below that each tile widens its
+ * codes in shared memory.  ZQ_OPT_GEMM_PATH = 3 forces the matrix-vector
+ * path (T <= 4), 4 the widening pass, 1 or 2 the in-tile widening;
+ * ZQ_OPT_CTA_PAIR = 2 forces 256-row units shared by a CTA pair (with the
+ * in-tile widening they measured slower and are never chosen automatically).
  * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
  * 16 <= K <= 2^20, K % 16 == 0, 1 <= g <= N, pointers 16-byte aligned.
  * Errors: as zq_gemm_w8a8 (argument errors before any launch).
@@ -264,9 +268,11 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  *                      3 = CUDA-core matrix-vector product (T <= 4, else
  *                          ZQ_ERR_UNSUPPORTED); automatic at T <= 4 with
  *                          INT4 weights and at T <= 2 with INT8 ones;
- *                      4 = INT4 weights widened into the workspace, then
- *                          the INT8 GEMM (zq_gemm_w4a8 only, else
- *                          ZQ_ERR_UNSUPPORTED); automatic at T >= 512.
+ *                      4 = the codes widened into the workspace first:
+ *                          zq_gemm_w4a8 then runs the INT8 GEMM (automatic
+ *                          at T >= 512), the FP16-activation GEMMs the fp16
+ *                          GEMM (automatic at T >= 1024); zq_gemm_w8a8
+ *                          returns ZQ_ERR_UNSUPPORTED.
  *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256);
  *                      the FP16-activation GEMMs accept 128 or 256 (other
  *                      values: ZQ_ERR_UNSUPPORTED) and ignore the path.
@@ -292,7 +298,8 @@ int zq_get_option(int key);
  * already), so that later GEMM calls of up to that need allocate nothing.
  * The need of a call: 4 * splits * T * N bytes for a split-K weight-streaming
  * plan, plus N * K bytes (rounded up to 256) when zq_gemm_w4a8 widens its
- * codes (T >= 512, or ZQ_OPT_GEMM_PATH = 4).  Synchronous; call it
+ * codes (T >= 512, or ZQ_OPT_GEMM_PATH = 4); 2 * N * K bytes when an
+ * FP16-activation GEMM widens its codes (T >= 1024, or path 4).  Synchronous; call it
  * outside stream capture.  Returns ZQ_ERR_CUDA if the allocation fails.
  */
 zq_status zq_workspace_reserve(unsigned long long bytes);

@@ -59,10 +59,15 @@ constexpr int tmem_cols_for(int v) {
   return p;
 }
 
-template <int BN_, bool W4_, bool PAIR_>
+template <int BN_, bool W4_, bool PAIR_, bool PRE_ = false>
 struct A16Cfg {
   static constexpr int BN = BN_;
   static constexpr bool W4 = W4_;
+  // PRE: the weights were widened to fp16 codes before the launch
+  // (widen_a16_kernel) and reach shared memory by TMA like the activations;
+  // the widening warps then have nothing to do.
+  static constexpr bool PRE = PRE_;
+  static_assert(!PRE || !W4, "pre-widened weights are fp16 whatever their code width");
   // CTA pair (cta_group::2): a 256 x BN tile per pair; each CTA holds 128
   // token rows of A, widens BN/2 weight rows of B, and keeps 128 rows of D.
   static constexpr bool PAIR = PAIR_;
@@ -71,7 +76,7 @@ struct A16Cfg {
   static constexpr int A_BYTES = kBM * 128;            // fp16 activations of one slice
   static constexpr int B_BYTES = B_ROWS * 128;         // widened weights of one slice
   static constexpr int CODE_ROW = W4 ? kKE / 2 : kKE;  // code bytes per weight row and slice
-  static constexpr int P_BYTES = B_ROWS * CODE_ROW;    // codes as stored in memory
+  static constexpr int P_BYTES = PRE ? 0 : B_ROWS * CODE_ROW;  // codes as stored in memory
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
   static constexpr int EPI_COLS = BN / 2;              // columns of one epilogue warp
   static constexpr int STG_BYTES = 32 * 32 * 2;        // one 32 x 32 fp16 output block
@@ -99,6 +104,7 @@ struct A16Cfg {
   static_assert(B_ROWS % 16 == 0, "widening steps of 16 rows keep each row's swizzle phase");
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(P_BYTES % 128 == 0, "TMA destination alignment");
+  static_assert(!PRE || B_ROWS <= 256, "one TMA box of weight rows");
   static_assert(EPI_COLS <= 128, "epilogue prefetch holds at most four columns per lane");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(TMEM_COLS <= 512, "TMEM accumulators");
@@ -255,7 +261,23 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             break;
           }
           // slices past K (and rows past T or N) read the TMA's zero fill
-          if constexpr (C::PAIR) {
+          if constexpr (C::PRE) {
+            // activations and fp16 weight rows, both in the MMA's layout; for
+            // a pair, both CTAs' tiles complete on the leader's full barrier
+            if constexpr (C::PAIR) {
+              const uint32_t fb = mapa_shared(smem_u32(&full_bar[stage]), 0);
+              if (crank == 0)
+                mbar_arrive_expect_tx(&full_bar[stage], 2u * (C::A_BYTES + C::B_BYTES));
+              tma_load_2d_pair(sA + stage * C::A_BYTES, &map_x, fb, kb * kKE, act_row, pol_x);
+              tma_load_2d_pair(sB + stage * C::B_BYTES, &map_w, fb, kb * kKE, w_row, pol_w);
+            } else {
+              mbar_arrive_expect_tx(&full_bar[stage], C::A_BYTES + C::B_BYTES);
+              tma_load_2d(sA + stage * C::A_BYTES, &map_x, &full_bar[stage], kb * kKE, act_row,
+                          pol_x);
+              tma_load_2d(sB + stage * C::B_BYTES, &map_w, &full_bar[stage], kb * kKE, w_row,
+                          pol_w);
+            }
+          } else if constexpr (C::PAIR) {
             // both CTAs' activation tiles complete on the leader's full
             // barrier (the MMA reads them); this CTA's codes on its own
             // pfull barrier (its widening warps read them)
@@ -285,7 +307,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       if (!C::PAIR || crank == 0)
         for (int s = 0; s < STAGES; ++s)
           if (fills[s]) mbar_wait(&full_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 22);
-      if (C::PAIR)
+      if (C::PAIR && !C::PRE)
         for (int s = 0; s < STAGES; ++s)
           if (fills[s]) mbar_wait(&pfull_bar[s], (fills[s] - 1) & 1, &no_abort, p.status, 28);
     }
@@ -306,8 +328,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
           // the widening warps arrive only after the stage's codes landed
           // (single CTA: with the activations, on the same barrier); a pair
           // also waits for both CTAs' activation tiles
-          if (!mbar_wait(&ready_bar[stage], phase, abort_flag, p.status, 24) ||
-              (C::PAIR && !mbar_wait(&full_bar[stage], phase, abort_flag, p.status, 29))) {
+          if ((!C::PRE && !mbar_wait(&ready_bar[stage], phase, abort_flag, p.status, 24)) ||
+              ((C::PAIR || C::PRE) && !mbar_wait(&full_bar[stage], phase, abort_flag, p.status, 29))) {
             ok = false;
             break;
           }
@@ -468,7 +490,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       }
       __syncwarp();
     }
-  } else {
+  } else if constexpr (!C::PRE) {
     // ------------------------------------------------------ widen the codes
     // Thread ut writes 16-byte chunk j = ut % 8 (eight k) of rows
     // r = ut / 8 + 16 i; stepping 16 rows keeps r % 8, so each thread's
@@ -534,7 +556,43 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
   }
 }
 
+// Codes widened once per call to exact fp16 integers [N][K] (the same bit
+// construction as the widening warps: the code, sign bit flipped, under the
+// exponent byte 0x64, minus 1024 + 128 or 1024 + 8).  HBM-bound: the codes
+// are read once and 2*N*K bytes written; the GEMM then reads the fp16 rows
+// by TMA, so no tile widens them again.
+template <bool W4>
+__global__ void __launch_bounds__(256)
+    widen_a16_kernel(const uint4* __restrict__ codes, uint4* __restrict__ wide, size_t n16) {
+  // the codes may be written by the previous kernel of the stream
+  grid_dependency_wait();
+  grid_launch_dependents();
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n16;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const uint4 w = __ldcs(codes + i);
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    if constexpr (W4) {  // 32 codes -> 64 bytes
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        uint32_t h[4];
+        widen8_i4(in[m], h);
+        wide[4 * i + m] = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+    } else {  // 16 codes -> 32 bytes
+      uint32_t h[8];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) widen4_i8(in[m], h[2 * m], h[2 * m + 1]);
+      wide[2 * i] = make_uint4(h[0], h[1], h[2], h[3]);
+      wide[2 * i + 1] = make_uint4(h[4], h[5], h[6], h[7]);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ host
+
+// From this many tokens the codes are widened once per call (widen_a16_kernel)
+// and the GEMM reads fp16 weights by TMA; below it the tiles widen them.
+constexpr int kA16WidenMinTokens = 1024;
 
 struct A16Plan {
   int bn, m_tiles, n_tiles, k_blocks, units;
@@ -611,11 +669,11 @@ cudaError_t launch_a16(const CUtensorMap& mx, const CUtensorMap& mw, const CUten
                     mw, my, p);
 }
 
-template <bool W4, bool PAIR>
+template <bool W4, bool PAIR, bool PRE = false>
 cudaError_t dispatch_a16(int bn, const CUtensorMap& mx, const CUtensorMap& mw,
                          const CUtensorMap& my, const A16Params& p, int grid, cudaStream_t st) {
-  return bn == 128 ? launch_a16<A16Cfg<128, W4, PAIR>>(mx, mw, my, p, grid, st)
-                   : launch_a16<A16Cfg<256, W4, PAIR>>(mx, mw, my, p, grid, st);
+  return bn == 128 ? launch_a16<A16Cfg<128, W4, PAIR, PRE>>(mx, mw, my, p, grid, st)
+                   : launch_a16<A16Cfg<256, W4, PAIR, PRE>>(mx, mw, my, p, grid, st);
 }
 
 zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_grp, int g,
@@ -643,12 +701,27 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   const int fbn = option(ZQ_OPT_GEMM_BN);
   if (fbn && fbn != 128 && fbn != 256) return ZQ_ERR_UNSUPPORTED;
   const int sms = num_sms();
-  // CTA pairs halve the widening and the weight-tile traffic per SM, but the
-  // cross-CTA handshake per stage costs more than that saves (measured on
-  // B200: GPT-NeoX QKV at T = 4096 1.67 ms with pairs, 1.39 ms without), so
-  // they run only when forced (ZQ_OPT_CTA_PAIR = 2)
-  const bool pair = option(ZQ_OPT_CTA_PAIR) == 2;
-  const A16Plan plan = plan_a16(T, N, K, sms, fbn, pair);
+  const int fpair = option(ZQ_OPT_CTA_PAIR);
+  // Prefill-sized token counts: widen the codes once (an HBM-bound pass into
+  // the library workspace), then a plain fp16 GEMM whose weight tiles arrive
+  // by TMA; ZQ_OPT_GEMM_PATH = 4 forces it.
+  const bool pre = forced_path == 4 || (forced_path == 0 && T >= kA16WidenMinTokens);
+  A16Plan plan;
+  if (pre) {
+    // with nothing to widen in the tiles, CTA pairs halve the weight-tile
+    // traffic per SM as in the INT8 GEMM: preferred for long rows
+    const A16Plan single = plan_a16(T, N, K, sms, fbn, false);
+    const A16Plan pr = plan_a16(T, N, K, sms, fbn, true);
+    plan = fpair == 1 ? single
+                      : (fpair == 2 || pr.cost * (K >= 2048 ? 0.82 : 1.10) < single.cost ? pr
+                                                                                      : single);
+  } else {
+    // In-tile widening: CTA pairs halve the widening and the weight-tile
+    // traffic per SM, but the cross-CTA handshake per stage costs more than
+    // that saves (measured on B200: GPT-NeoX QKV at T = 4096 1.67 ms with
+    // pairs, 1.39 ms without), so they run only when forced
+    plan = plan_a16(T, N, K, sms, fbn, fpair == 2);
+  }
 
   int* status = device_status_ptr();
   if (!status) return ZQ_ERR_CUDA;
@@ -671,11 +744,30 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   // in 32 x 32 blocks.
   const int code_row = w4 ? kKE / 2 : kKE;
   const uint64_t w_inner = w4 ? static_cast<uint64_t>(K) / 2 : static_cast<uint64_t>(K);
+  const int w_box_rows = plan.pair ? plan.bn / 2 : plan.bn;
+  const void* wsrc = Wq;
+  if (pre) {
+    void* wide = nullptr;
+    if (library_workspace(static_cast<size_t>(N) * K * 2, &wide) != cudaSuccess)
+      return ZQ_ERR_CUDA;
+    const size_t n16 = static_cast<size_t>(N) * w_inner / 16;
+    const int blocks = static_cast<int>(std::min<size_t>((n16 + 255) / 256, 8 * sms));
+    const cudaError_t we =
+        w4 ? launch_pdl(widen_a16_kernel<true>, dim3(std::max(blocks, 1)), dim3(256), 0, st,
+                        static_cast<const uint4*>(Wq), static_cast<uint4*>(wide), n16)
+           : launch_pdl(widen_a16_kernel<false>, dim3(std::max(blocks, 1)), dim3(256), 0, st,
+                        static_cast<const uint4*>(Wq), static_cast<uint4*>(wide), n16);
+    if (we != cudaSuccess) return ZQ_ERR_CUDA;
+    wsrc = wide;
+  }
   CUtensorMap mx, mw, my;
   if (!encode_tma_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, K, T, static_cast<uint64_t>(K) * 2,
                      kKE, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, Wq, w_inner, N, w_inner, code_row,
-                     plan.pair ? plan.bn / 2 : plan.bn, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !(pre ? encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wsrc, K, N,
+                            static_cast<uint64_t>(K) * 2, kKE, w_box_rows,
+                            CU_TENSOR_MAP_SWIZZLE_128B)
+            : encode_tma_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, wsrc, w_inner, N, w_inner,
+                            code_row, w_box_rows, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
       !encode_tma_2d(&my, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Y, N, T, static_cast<uint64_t>(N) * 2,
                      32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return ZQ_ERR_CUDA;
@@ -688,7 +780,10 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
     if (cap > 0) grid = std::min(grid, std::max(2, cap & ~1));
   }
   cudaError_t e;
-  if (plan.pair)
+  if (pre)
+    e = plan.pair ? dispatch_a16<false, true, true>(plan.bn, mx, mw, my, p, grid, st)
+                  : dispatch_a16<false, false, true>(plan.bn, mx, mw, my, p, grid, st);
+  else if (plan.pair)
     e = w4 ? dispatch_a16<true, true>(plan.bn, mx, mw, my, p, grid, st)
            : dispatch_a16<false, true>(plan.bn, mx, mw, my, p, grid, st);
   else

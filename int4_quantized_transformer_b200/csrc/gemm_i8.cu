@@ -1036,6 +1036,17 @@ cudaError_t ensure_workspace(size_t elems, Workspace** out) {
   return cudaSuccess;
 }
 
+}  // namespace
+
+cudaError_t library_workspace(size_t bytes, void** out) {
+  Workspace* w = nullptr;
+  const cudaError_t e = ensure_workspace((bytes + 3) / 4, &w);
+  if (e == cudaSuccess) *out = w->ws;
+  return e;
+}
+
+namespace {
+
 // The split-K finalisation, launched right after the GEMM kernel on the same
 // stream (programmatic dependent launch: it is scheduled early and waits in
 // the kernel for the GEMM's partial sums).

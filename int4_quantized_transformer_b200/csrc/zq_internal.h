@@ -33,6 +33,11 @@ cudaError_t launch_gemv_a16(int bits, const void* X, const void* W, const float*
                             const void* bias, int T, int N, int K, void* Y, float* acc_dbg,
                             int max_ctas, cudaStream_t st);
 int option(int key);
+// The library workspace of the current device (gemm_i8.cu): at least
+// `bytes` bytes, grown with cudaMalloc when a call needs more than it holds.
+// One buffer per device; calls that use it on different streams must not
+// overlap.
+cudaError_t library_workspace(size_t bytes, void** out);
 // Counts one kernel launch issued by the library (zq_launch_count).
 void count_launch();
 

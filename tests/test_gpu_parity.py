@@ -540,6 +540,17 @@ def test_gemm_a16_gemv_path(zq, bits, T, N, K, g):
     _check_a16(zq, T, N, K, g, bits, seed=T * 7 + N + 1, bias=False, path=3, max_ctas=5)
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("pair", [1, 2])
+@pytest.mark.parametrize("T,N,K", [(16, 256, 64), (513, 1000, 256), (1024, 768, 1024),
+                                   (700, 2304, 448), (1100, 520, 2112)])
+def test_gemm_a16_widened_weights(zq, bits, pair, T, N, K):
+    """Codes widened once into fp16 rows in the workspace, then the fp16 GEMM
+    with TMA-fed weight tiles (automatic from 1024 tokens, forced here), on
+    single CTAs and CTA pairs."""
+    _check_a16(zq, T, N, K, 8, bits, seed=T + N + pair, path=4, pair=pair)
+
+
 def test_gemm_a16_small_t_on_tensor_cores(zq):
     """The tensor-core path forced for a few tokens (one partial 128-row tile)."""
     _check_a16(zq, 3, 520, 256, 8, 8, seed=41, path=1)

@@ -567,9 +567,7 @@ __global__ void __launch_bounds__(256)
   // the codes may be written by the previous kernel of the stream
   grid_dependency_wait();
   grid_launch_dependents();
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n16;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint4 w = __ldcs(codes + i);
+  auto one = [&](uint4 w, size_t i) {
     const uint32_t in[4] = {w.x, w.y, w.z, w.w};
     if constexpr (W4) {  // 32 codes -> 64 bytes
 #pragma unroll
@@ -585,7 +583,19 @@ __global__ void __launch_bounds__(256)
       wide[2 * i] = make_uint4(h[0], h[1], h[2], h[3]);
       wide[2 * i + 1] = make_uint4(h[4], h[5], h[6], h[7]);
     }
+  };
+  // four 16-byte loads in flight per thread, so the pass runs at the HBM rate
+  constexpr int U = 4;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  for (; i + (U - 1) * stride < n16; i += U * stride) {
+    uint4 w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) w[u] = __ldcs(codes + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < U; ++u) one(w[u], i + u * stride);
   }
+  for (; i < n16; i += stride) one(__ldcs(codes + i), i);
 }
 
 // ------------------------------------------------------------------ host

@@ -57,6 +57,7 @@ constexpr int BK = 128;       // K bytes per pipeline stage (one swizzle row)
 constexpr int UMMA_K = 32;    // K of one tcgen05.mma kind::i8
 constexpr int kSmemBudget = 223 * 1024;
 constexpr int NUM_EPI_WARPS_C = 8;
+constexpr int kTmemUnpackWarps = 4;
 
 constexpr int pow2_at_least(int v) {
   int p = 32;
@@ -134,7 +135,10 @@ struct Cfg {
   static constexpr int TMEM_COLS =
       pow2_at_least(2 * BUF_COLS + (TMEM_A ? STAGES * 32 * KPS : 0));
   static constexpr int NUM_EPI_WARPS = NUM_EPI_WARPS_C;
-  static constexpr int NUM_UNPACK_WARPS = W4 ? 4 : 0;
+  // INT4 unpack warps: four (one per TMEM lane quadrant); with the TMEM
+  // operand ring, kTmemUnpackWarps of them (eight: two per quadrant, each
+  // widening one of the stage's two K slices)
+  static constexpr int NUM_UNPACK_WARPS = W4 ? (TMEM_A ? kTmemUnpackWarps : 4) : 0;
   static constexpr int NUM_WARPS = 1 + NUM_PROD_WARPS + NUM_EPI_WARPS + NUM_UNPACK_WARPS;
   static constexpr int NUM_THREADS = 32 * NUM_WARPS;
   // shared memory carve-up (offsets from a 1024-byte aligned base)
@@ -840,8 +844,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
             const uint8_t* prow = sP + pst * C::P_BYTES + r * PROW;
             const uint32_t a_tm = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
                                   static_cast<uint32_t>(C::A_COL0 + stage * C::KPS * 32);
+            // with two warps per quadrant, each widens one K slice of the stage
+            constexpr int HPW = C::NUM_UNPACK_WARPS >= 4 * C::KPS ? 1 : C::KPS;  // slices per warp
+            const int hb = HPW == 1 ? (ut / 128) : 0;
 #pragma unroll
-            for (int h = 0; h < C::KPS; ++h) {
+            for (int h = hb; h < hb + HPW; ++h) {
               uint32_t w[32];
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
@@ -988,24 +995,37 @@ __device__ __forceinline__ uint32_t sext_nibbles(uint32_t n) {
   return n | ((n & 0x08080808u) * 0x1Eu);
 }
 
+constexpr int kWidenUnroll = 4;  // 16-byte loads in flight per thread
+
+__device__ __forceinline__ void widen_store(uint4 w, uint4* dst) {
+  const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+  uint32_t out[8];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    out[2 * m] = sext_nibbles(in[m] & 0x0F0F0F0Fu);             // k = 8m .. 8m + 3
+    out[2 * m + 1] = sext_nibbles((in[m] >> 4) & 0x0F0F0F0Fu);  // k = 8m + 4 .. 8m + 7
+  }
+  dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+  dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
 __global__ void __launch_bounds__(256)
     widen_w4_kernel(const uint4* __restrict__ packed, uint4* __restrict__ wide, size_t n16) {
   // the packed codes may be written by the previous kernel of the stream
   grid_dependency_wait();
   grid_launch_dependents();
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n16;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const uint4 w = __ldcs(packed + i);  // 32 codes: k = 32i .. 32i + 31 of one row
-    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-    uint32_t out[8];
+  // each thread keeps kWidenUnroll loads in flight (a 16-byte chunk = 32
+  // codes: k = 32i .. 32i + 31 of one row), so the pass runs at the HBM rate
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  for (; i + (kWidenUnroll - 1) * stride < n16; i += kWidenUnroll * stride) {
+    uint4 w[kWidenUnroll];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      out[2 * m] = sext_nibbles(in[m] & 0x0F0F0F0Fu);             // k = 8m .. 8m + 3
-      out[2 * m + 1] = sext_nibbles((in[m] >> 4) & 0x0F0F0F0Fu);  // k = 8m + 4 .. 8m + 7
-    }
-    wide[2 * i] = make_uint4(out[0], out[1], out[2], out[3]);
-    wide[2 * i + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+    for (int u = 0; u < kWidenUnroll; ++u) w[u] = __ldcs(packed + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < kWidenUnroll; ++u) widen_store(w[u], wide + 2 * (i + u * stride));
   }
+  for (; i < n16; i += stride) widen_store(__ldcs(packed + i), wide + 2 * i);
 }
 
 // ------------------------------------------------------------------ host
@@ -1443,6 +1463,8 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   if (ch.widen) {
     const size_t n16 = static_cast<size_t>(N) * (K / 2) / 16;
     const int blocks = static_cast<int>(std::min<size_t>((n16 + 255) / 256, 8 * num_sms()));
+    // (8 resident CTAs of 256 threads per SM, each thread kWidenUnroll
+    // chunks in flight)
     if (launch_pdl(widen_w4_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, st,
                    static_cast<const uint4*>(Wq), reinterpret_cast<uint4*>(ws), n16) != cudaSuccess)
       return ZQ_ERR_CUDA;

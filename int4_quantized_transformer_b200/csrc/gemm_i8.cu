@@ -179,6 +179,13 @@ struct GemmParams {
   int T, N, K, g;
   int m_tiles, n_tiles, k_blocks, splits, num_units;
   int kps;  // K slices per pipeline stage (Cfg::KPS of the launched kernel)
+  // Token-row tiling with a short last wave: the tiles from tail_start on
+  // are split along K into tail_splits parts of tail_kb K slices each; their
+  // exact int32 partial sums go to ws (tail tile j, part s at
+  // ws + (j * tail_splits + s) * TILE_M * BN, row-major) and
+  // tail_finalize_kernel adds them and dequantizes.  tail_start = the number
+  // of tiles when there is no tail.
+  int tail_start, tail_splits, tail_kb;
   // unit order: 0 = M tiles fastest (consecutive units, which run at the
   // same time, share their N-side operand tile), 1 = N tiles fastest
   int n_fastest;
@@ -194,10 +201,24 @@ struct GemmParams {
 // which the DRAM serves as longer contiguous runs than S separate ranges.
 struct Unit {
   int m, n, kb0, kb1, kstep, split;
+  int tail;  // index among the split tiles of the last wave, or -1
 };
 
 __device__ __forceinline__ Unit decode_unit(int u, const GemmParams& p) {
   Unit r;
+  r.tail = -1;
+  if (u >= p.tail_start) {  // a K part of a last-wave token-row tile
+    const int j = u - p.tail_start;
+    const int rest = p.tail_start + j / p.tail_splits;
+    r.tail = j / p.tail_splits;
+    r.split = j % p.tail_splits;
+    r.m = rest % p.m_tiles;
+    r.n = rest / p.m_tiles;
+    r.kb0 = r.split * p.tail_kb;
+    r.kb1 = min(p.k_blocks, r.kb0 + p.tail_kb);
+    r.kstep = p.kps;
+    return r;
+  }
   const int split = u % p.splits;
   const int rest = u / p.splits;
   if (p.n_fastest) {
@@ -605,6 +626,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
       }
       if (u >= p.num_units || split) return;
       const Unit t = decode_unit(u, p);
+      if (t.tail >= 0) return;  // a last-wave K part stores raw partial sums
       if (C::WROWS) {
         const int o = t.m * BM + row_in_tile;
         if (o < p.N) {
@@ -774,6 +796,24 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
               a0[j] = static_cast<uint32_t>(static_cast<int>(a0[j]) >> 4);
               a1[j] = static_cast<uint32_t>(static_cast<int>(a1[j]) >> 4);
             }
+          }
+          if (!C::WROWS && t.tail >= 0) {
+            // a K part of a last-wave tile: the exact int32 partial sums of
+            // this lane's token row, 32 columns at a time (finalized by
+            // tail_finalize_kernel)
+            int32_t* prow = p.ws + (static_cast<size_t>(t.tail * p.tail_splits + t.split) * C::TILE_M +
+                                    static_cast<int>(crank) * BM + row_in_tile) * BN + c0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              reinterpret_cast<uint4*>(prow)[q] =
+                  make_uint4(a0[4 * q], a0[4 * q + 1], a0[4 * q + 2], a0[4 * q + 3]);
+            if (two) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                reinterpret_cast<uint4*>(prow + 32)[q] =
+                    make_uint4(a1[4 * q], a1[4 * q + 1], a1[4 * q + 2], a1[4 * q + 3]);
+            }
+            continue;
           }
           uint32_t h[16];
           dequant_tok(a0, c0, h);
@@ -978,6 +1018,63 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The last-wave tiles of the token-row tiling, split along K: add each
+// output's int32 partial sums (exact) and dequantize, eight outputs per
+// thread, y = fp16(((f32(acc) * s_tok[t]) * s_grp[group(o)]) + f32(bias[o])).
+// Partials of tail tile j, part s: ws + (j * splits + s) * tile_m * bn,
+// row-major [tile_m][bn].
+__global__ void __launch_bounds__(256)
+    tail_finalize_kernel(const int32_t* __restrict__ ws, int ntail, int splits, int tail_start,
+                         int m_tiles, int tile_m, int bn, const float* __restrict__ s_tok,
+                         const float* __restrict__ s_grp, const __half* __restrict__ bias,
+                         __half* __restrict__ Y, int32_t* __restrict__ acc_dbg, int T, int N,
+                         int g) {
+  // the partial sums are written by the GEMM kernel just before this one
+  grid_dependency_wait();
+  grid_launch_dependents();
+  const size_t tile_elems = static_cast<size_t>(tile_m) * bn;
+  const size_t n8 = static_cast<size_t>(ntail) * tile_elems / 8;  // bn % 8 == 0
+  for (size_t v = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; v < n8;
+       v += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t e = v * 8;
+    const int j = static_cast<int>(e / tile_elems);
+    const int within = static_cast<int>(e - static_cast<size_t>(j) * tile_elems);
+    const int lrow = within / bn, lcol = within - lrow * bn;
+    const int tile = tail_start + j;
+    const int t = (tile % m_tiles) * tile_m + lrow;
+    const int o = (tile / m_tiles) * bn + lcol;
+    if (t >= T || o >= N) continue;  // N % 8 == 0: eight columns are all in or all out
+    const int32_t* src = ws + static_cast<size_t>(j) * splits * tile_elems + within;
+    int4 lo = __ldcg(reinterpret_cast<const int4*>(src));
+    int4 hi = __ldcg(reinterpret_cast<const int4*>(src) + 1);
+    for (int sp = 1; sp < splits; ++sp) {
+      const int4* q = reinterpret_cast<const int4*>(src + sp * tile_elems);
+      const int4 a = __ldcg(q), b = __ldcg(q + 1);
+      lo.x += a.x; lo.y += a.y; lo.z += a.z; lo.w += a.w;
+      hi.x += b.x; hi.y += b.y; hi.z += b.z; hi.w += b.w;
+    }
+    const int acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    const float st = __ldg(s_tok + t);
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 8; q += 2) {
+      float v0 = __fmul_rn(__int2float_rn(acc[q]), st);
+      float v1 = __fmul_rn(__int2float_rn(acc[q + 1]), st);
+      v0 = __fadd_rn(__fmul_rn(v0, __ldg(s_grp + group_of(o + q, N, g))),
+                     bias ? __half2float(bias[o + q]) : 0.0f);
+      v1 = __fadd_rn(__fmul_rn(v1, __ldg(s_grp + group_of(o + q + 1, N, g))),
+                     bias ? __half2float(bias[o + q + 1]) : 0.0f);
+      h[q / 2] = pack_half2(v0, v1);
+    }
+    const size_t idx = static_cast<size_t>(t) * N + o;
+    *reinterpret_cast<uint4*>(Y + idx) = make_uint4(h[0], h[1], h[2], h[3]);
+    if (acc_dbg) {
+      reinterpret_cast<int4*>(acc_dbg + idx)[0] = lo;
+      reinterpret_cast<int4*>(acc_dbg + idx)[1] = hi;
+    }
+  }
+}
+
 // INT4 weights for prefill-sized token counts: the packed codes are widened
 // once per call to int8 codes in a workspace, [N][K] in k order, and the
 // INT8 GEMM reads them from there.  Each weight tile is then widened once
@@ -1084,6 +1181,10 @@ struct Plan {
   int bn;
   int m_tiles, n_tiles, k_blocks, splits, kb_per_split, units;
   int kps = 1;  // K slices per pipeline stage (weight rows with INT4 weights: 2)
+  // token rows: tiles from tail_start on (the last, short wave) are split
+  // along K into tail_splits parts of tail_kb slices (tail_start = the tile
+  // count when there is no such split)
+  int tail_start = 0, tail_splits = 1, tail_kb = 0;
   double cost;
 };
 
@@ -1158,7 +1259,7 @@ Plan plan_wrows(int T, int N, int K, int sms, int forced_split, bool w4) {
 // Token-row tiling: 128 x BN tiles per CTA, or 256 x BN tiles per CTA pair
 // (each CTA of the pair does the same MMA work as a single-CTA tile, so a
 // unit costs the same; there are half as many "slots").
-Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair) {
+Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair, bool allow_tail) {
   Plan best{};
   best.cost = 1e30;
   const int cands[3] = {256, 192, 128};
@@ -1175,8 +1276,23 @@ Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair) {
     p.splits = 1;
     p.kb_per_split = p.k_blocks;
     p.units = p.m_tiles * p.n_tiles;
+    p.tail_start = p.units;
     const int waves = ceil_div(p.units, slots);
     p.cost = waves * (p.k_blocks * 2.0 * bn + 600.0);
+    // A last wave less than half full: split its tiles along K over the idle
+    // slots (parts of at least four K slices), so that wave takes a fraction
+    // of a tile's time; a finalize kernel adds the parts.
+    const int full = p.units / slots, rem = p.units % slots;
+    if (allow_tail && full >= 1 && rem > 0 && 2 * rem <= slots) {
+      const int want = std::min(std::min(slots / rem, p.k_blocks / 4), 8);
+      if (want >= 2) {
+        p.tail_kb = ceil_div(p.k_blocks, want);
+        p.tail_splits = ceil_div(p.k_blocks, p.tail_kb);
+        p.tail_start = full * slots;
+        p.units = p.tail_start + rem * p.tail_splits;
+        p.cost = full * (p.k_blocks * 2.0 * bn + 600.0) + (p.tail_kb * 2.0 * bn + 600.0) + 400.0;
+      }
+    }
     if (p.cost < best.cost) best = p;
   }
   return best;
@@ -1293,7 +1409,8 @@ struct Choice {
 // 123 us), the pass then being a third of the time.
 constexpr int kWidenMinTokens = 512;
 
-zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
+zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out,
+                 bool allow_tail = true) {
   const int sms = num_sms();
   // A handful of tokens: the CUDA-core matrix-vector path (measured faster
   // than the tensor-core tilings up to T = 4 with INT4 weights and up to
@@ -1327,12 +1444,12 @@ zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
   // tiles run ~18% faster per tile when K >= 2048 and ~10% slower at small
   // K, so the two wave-aware plans are compared with those factors.
   const int fpair = option(ZQ_OPT_CTA_PAIR);
-  const Plan single = plan_trows(T, N, K, sms, fbn, false);
+  const Plan single = plan_trows(T, N, K, sms, fbn, false, allow_tail);
   if (fpair == 1) {
     out->plan = single;
     return ZQ_OK;
   }
-  const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true);
+  const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true, allow_tail);
   // INT4: the unpack stage, not the operand feed, bounds the mainloop;
   // pairs measured slower there, so they are used only when forced.
   const double f = w4 ? 1e9 : (K >= 2048 ? 0.82 : 1.10);
@@ -1340,9 +1457,29 @@ zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out) {
   return ZQ_OK;
 }
 
-// Partial sums a weight-row plan with K splits stores (int32 elements).
+// Last-wave tiles a token-row plan splits along K.
+int tail_tiles(const Plan& plan) {
+  return plan.wrows ? 0 : (plan.units - plan.tail_start) / plan.tail_splits;
+}
+
+// Partial sums a plan stores (int32 elements): a weight-row plan with K
+// splits, or the K parts of a token-row plan's last-wave tiles.
 size_t split_partials(const Plan& plan, int T, int N) {
-  return (plan.wrows && plan.splits > 1) ? static_cast<size_t>(plan.splits) * T * N : 0;
+  if (plan.wrows) return plan.splits > 1 ? static_cast<size_t>(plan.splits) * T * N : 0;
+  return static_cast<size_t>(tail_tiles(plan)) * plan.tail_splits * (plan.pair ? 2 * BM : BM) *
+         plan.bn;
+}
+
+// The finalisation of the last-wave tiles, chained after the GEMM kernel.
+cudaError_t launch_tail_finalize(const GemmParams& gp, const Plan& plan, cudaStream_t st) {
+  const int ntail = tail_tiles(plan);
+  const int tile_m = plan.pair ? 2 * BM : BM;
+  const size_t n8 = static_cast<size_t>(ntail) * tile_m * plan.bn / 8;
+  const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 4 * 148));
+  return launch_pdl(tail_finalize_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, st,
+                    static_cast<const int32_t*>(gp.ws), ntail, plan.tail_splits, plan.tail_start,
+                    gp.m_tiles, tile_m, plan.bn, gp.s_tok, gp.s_grp, gp.bias, gp.Y, gp.acc_dbg, gp.T,
+                    gp.N, gp.g);
 }
 
 // Launches a chosen plan; `ws` receives the split-K partial sums (at least
@@ -1377,6 +1514,9 @@ zq_status launch_choice(bool w4, const Choice& ch, const int8_t* Xq, const float
   gp.splits = plan.splits;
   gp.kps = plan.kps;
   gp.num_units = plan.units;
+  gp.tail_start = plan.wrows ? plan.units : plan.tail_start;
+  gp.tail_splits = plan.tail_splits;
+  gp.tail_kb = plan.tail_kb;
   // Weight rows with several token tiles: when the weights are the larger
   // operand, let the CTAs running at the same time share a weight tile (each
   // weight tile then comes from DRAM once, the activations from L2).
@@ -1436,7 +1576,8 @@ zq_status launch_choice(bool w4, const Choice& ch, const int8_t* Xq, const float
   else
     e = w4 ? dispatch_bn<false, true>(plan.bn, ma, mw, my, gp, grid, st)
            : dispatch_bn<false, false>(plan.bn, ma, mw, my, gp, grid, st);
-  if (e == cudaSuccess && split_partials(plan, T, N) > 0) e = launch_finalize(gp, st);
+  if (e == cudaSuccess && split_partials(plan, T, N) > 0)
+    e = plan.wrows ? launch_finalize(gp, st) : launch_tail_finalize(gp, plan, st);
   return e == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
 }
 
@@ -1554,6 +1695,11 @@ extern "C" zq_status zq_gemm_w8a8_noalloc(const int8_t* Xq, const float* s_tok, 
   Choice ch;
   rc = choose(false, T, N, K, forced_split, &ch);
   if (rc != ZQ_OK) return rc;
+  if (!ch.gemv && !ch.plan.wrows && split_partials(ch.plan, T, N) > kNoAllocPartialInts) {
+    // a token-row plan whose last-wave split does not fit: plan without it
+    rc = choose(false, T, N, K, forced_split, &ch, false);
+    if (rc != ZQ_OK) return rc;
+  }
   if (!ch.gemv && split_partials(ch.plan, T, N) > kNoAllocPartialInts) {
     if (forced_split > 0) return ZQ_ERR_SHAPE;
     const size_t fit = kNoAllocPartialInts / (static_cast<size_t>(T) * N);

@@ -239,6 +239,16 @@ def test_gemm_cta_pair_tiles(zq, bits, bn, T, N, K):
 
 
 @pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("T,N,K,pair", [(2560, 2048, 1024, 2), (2048, 2560, 2048, 1),
+                                        (2600, 2056, 1056, 2)])
+def test_gemm_last_wave_split(zq, bits, T, N, K, pair):
+    """A last wave less than half full: its tiles are split along K, their int32
+    partial sums added and dequantized by the finalize kernel (80 pair units
+    over 74 pair slots, 160 single-CTA units over 148 SMs; ragged T, N and K)."""
+    _check_gemm(zq, T, N, K, 8, bits, seed=T + K + pair, pair=pair)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("split", [1, 2, 3, 7])
 @pytest.mark.parametrize("T,N,K", [(1, 512, 1024), (8, 1024, 896), (64, 384, 2048),
                                    (200, 256, 1024), (300, 256, 512)])

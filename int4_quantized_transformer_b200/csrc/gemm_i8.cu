@@ -1281,16 +1281,20 @@ Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair, bool all
     p.cost = waves * (p.k_blocks * 2.0 * bn + 600.0);
     // A last wave less than half full: split its tiles along K over the idle
     // slots (parts of at least four K slices), so that wave takes a fraction
-    // of a tile's time; a finalize kernel adds the parts.
+    // of a tile's time; a finalize kernel adds the parts.  Only 256-wide
+    // tiles: narrower ones cost more per MAC than the cost model counts
+    // (measured on B200: 256 x 192 and 256 x 128 CTA-pair tiles 1.1x and
+    // 1.5x the time per MAC of 256 x 256 ones), and the finalize launch is
+    // charged about 2 us.
     const int full = p.units / slots, rem = p.units % slots;
-    if (allow_tail && full >= 1 && rem > 0 && 2 * rem <= slots) {
+    if (allow_tail && bn == 256 && full >= 1 && rem > 0 && 2 * rem <= slots) {
       const int want = std::min(std::min(slots / rem, p.k_blocks / 4), 8);
       if (want >= 2) {
         p.tail_kb = ceil_div(p.k_blocks, want);
         p.tail_splits = ceil_div(p.k_blocks, p.tail_kb);
         p.tail_start = full * slots;
         p.units = p.tail_start + rem * p.tail_splits;
-        p.cost = full * (p.k_blocks * 2.0 * bn + 600.0) + (p.tail_kb * 2.0 * bn + 600.0) + 400.0;
+        p.cost = full * (p.k_blocks * 2.0 * bn + 600.0) + (p.tail_kb * 2.0 * bn + 600.0) + 4000.0;
       }
     }
     if (p.cost < best.cost) best = p;

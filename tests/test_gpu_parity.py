@@ -245,7 +245,7 @@ def test_gemm_last_wave_split(zq, bits, T, N, K, pair):
     """A last wave less than half full: its tiles are split along K, their int32
     partial sums added and dequantized by the finalize kernel (80 pair units
     over 74 pair slots, 160 single-CTA units over 148 SMs; ragged T, N and K)."""
-    _check_gemm(zq, T, N, K, 8, bits, seed=T + K + pair, pair=pair)
+    _check_gemm(zq, T, N, K, 8, bits, seed=T + K + pair, pair=pair, bn=256)
 
 
 @pytest.mark.parametrize("bits", [8, 4])

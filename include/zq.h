@@ -179,6 +179,22 @@ zq_status zq_gemm_w4a8(const int8_t* Xq, const float* s_tok, const uint8_t* Wq4,
                        int32_t* acc_dbg, zq_stream_t stream);
 
 /*
+ * zq_widen_int4_weights -- the INT4 unpack step on its own (Sec. 3.4 "Which
+ * weights get INT4": INT4 weights are converted to INT8 before the INT8
+ * GEMM): packed codes to int8 codes, an HBM-bound pass.  zq_gemm_w4a8 runs
+ * it itself at prefill token counts; calling it separately lets a caller
+ * widen a layer's INT4 weights ahead of time, for example on a second
+ * stream while other GEMMs run, and then call zq_gemm_w8a8 on the result
+ * (which gives the same outputs as zq_gemm_w4a8).
+ *   Wq4    uint8 [N][K/2] in the layout of zq_quantize_weights_groupwise(bits=4).
+ *   Wq8    int8 [N][K] output, caller-owned: Wq8[o][k] = the signed code of
+ *          weight (o, k), in -8..7 (-8 never occurs in quantized weights).
+ * Requirements: N >= 1, K >= 32, K % 32 == 0, pointers 16-byte aligned.
+ * Asynchronous on `stream`; argument errors return before any launch.
+ */
+zq_status zq_widen_int4_weights(const uint8_t* Wq4, int N, int K, int8_t* Wq8, zq_stream_t stream);
+
+/*
  * zq_gemm_w8a16 -- the quantized linear layer with FP16 activations and
  * group-wise INT8 weights (W8A16: the summary page's "Main Quantitative
  * Results", Table 4; also the GPT-NeoX self-attention input that stays in
@@ -276,7 +292,10 @@ zq_status zq_device_status(zq_stream_t stream, int* detail);
  *   ZQ_OPT_GEMM_BN     MMA N tile width for path 1 (a multiple of 16, 16..256);
  *                      the FP16-activation GEMMs accept 128 or 256 (other
  *                      values: ZQ_ERR_UNSUPPORTED) and ignore the path.
- *   ZQ_OPT_SPLIT_K     number of K splits for path 2 (1 = none).
+ *   ZQ_OPT_SPLIT_K     number of K splits for path 2 (1 = none); for path 1,
+ *                      the number of K parts of each tile of a partial last
+ *                      wave (automatic: for rows of K >= 12288 when that
+ *                      wave is less than half full).
  *   ZQ_OPT_MAX_CTAS    cap on the number of CTAs of the GEMM (persistent grid).
  *   ZQ_OPT_CTA_PAIR    path 1: 1 = one CTA per 128 x BN
  *                      tile, 2 = CTA pairs sharing 256 x BN tiles (tcgen05

@@ -1259,7 +1259,8 @@ Plan plan_wrows(int T, int N, int K, int sms, int forced_split, bool w4) {
 // Token-row tiling: 128 x BN tiles per CTA, or 256 x BN tiles per CTA pair
 // (each CTA of the pair does the same MMA work as a single-CTA tile, so a
 // unit costs the same; there are half as many "slots").
-Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair, bool allow_tail) {
+Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair, bool allow_tail,
+                int forced_tail) {
   Plan best{};
   best.cost = 1e30;
   const int cands[3] = {256, 192, 128};
@@ -1286,9 +1287,17 @@ Plan plan_trows(int T, int N, int K, int sms, int forced_bn, bool pair, bool all
     // (measured on B200: 256 x 192 and 256 x 128 CTA-pair tiles 1.1x and
     // 1.5x the time per MAC of 256 x 256 ones), and the finalize launch is
     // charged about 2 us.
+    // Measured on GPT-NeoX at T = 4096: FFN2 (K = 24576) 449 -> 401 us with the
+    // split, attention-out (K = 6144) unchanged (its finalize cost what the
+    // shorter wave saved), so it is automatic for long rows only;
+    // ZQ_OPT_SPLIT_K > 1 forces it (that many parts) whenever the last wave
+    // is partial.
     const int full = p.units / slots, rem = p.units % slots;
-    if (allow_tail && bn == 256 && full >= 1 && rem > 0 && 2 * rem <= slots) {
-      const int want = std::min(std::min(slots / rem, p.k_blocks / 4), 8);
+    const bool forced = forced_tail > 1 && rem > 0 && full >= 1;
+    if (allow_tail && (forced || (bn == 256 && p.k_blocks >= 96 && full >= 1 && rem > 0 &&
+                                  2 * rem <= slots))) {
+      const int want = forced ? std::min(forced_tail, p.k_blocks)
+                              : std::min(std::min(slots / rem, p.k_blocks / 4), 8);
       if (want >= 2) {
         p.tail_kb = ceil_div(p.k_blocks, want);
         p.tail_splits = ceil_div(p.k_blocks, p.tail_kb);
@@ -1448,12 +1457,12 @@ zq_status choose(bool w4, int T, int N, int K, int forced_split, Choice* out,
   // tiles run ~18% faster per tile when K >= 2048 and ~10% slower at small
   // K, so the two wave-aware plans are compared with those factors.
   const int fpair = option(ZQ_OPT_CTA_PAIR);
-  const Plan single = plan_trows(T, N, K, sms, fbn, false, allow_tail);
+  const Plan single = plan_trows(T, N, K, sms, fbn, false, allow_tail, forced_split);
   if (fpair == 1) {
     out->plan = single;
     return ZQ_OK;
   }
-  const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true, allow_tail);
+  const Plan pr = plan_trows(T, N, K, sms, fbn ? fbn : 256, true, allow_tail, forced_split);
   // INT4: the unpack stage, not the operand feed, bounds the mainloop;
   // pairs measured slower there, so they are used only when forced.
   const double f = w4 ? 1e9 : (K >= 2048 ? 0.82 : 1.10);
@@ -1621,6 +1630,21 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
 
 }  // namespace
 }  // namespace zq
+
+extern "C" zq_status zq_widen_int4_weights(const uint8_t* Wq4, int N, int K, int8_t* Wq8,
+                                           zq_stream_t stream) {
+  using namespace zq;
+  if (N < 1 || K < 32 || K % 32 != 0) return ZQ_ERR_SHAPE;
+  if (!Wq4 || !Wq8) return ZQ_ERR_NULL;
+  if (!aligned16(Wq4) || !aligned16(Wq8)) return ZQ_ERR_ALIGN;
+  const size_t n16 = static_cast<size_t>(N) * (K / 2) / 16;
+  const int blocks = static_cast<int>(std::min<size_t>((n16 + 255) / 256, 8 * num_sms()));
+  if (launch_pdl(widen_w4_kernel, dim3(std::max(blocks, 1)), dim3(256), 0,
+                 reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<const uint4*>(Wq4),
+                 reinterpret_cast<uint4*>(Wq8), n16) != cudaSuccess)
+    return ZQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+}
 
 extern "C" zq_status zq_workspace_reserve(unsigned long long bytes) {
   zq::Workspace* w = nullptr;

@@ -25,6 +25,7 @@ EXPORTS = (
     "zq_gemm_w8a8", "zq_gemm_w4a8", "zq_device_status", "zq_set_option", "zq_get_option",
     "zq_debug_wait_timeout", "zq_gemm_w8a8_noalloc", "zq_bias_act_quant", "zq_static_quant",
     "zq_gemm_w8a16", "zq_gemm_w4a16", "zq_launch_count", "zq_workspace_reserve",
+    "zq_widen_int4_weights",
 )
 
 
@@ -58,6 +59,7 @@ def _load():
         "zq_gemm_w4a16": ([P, P, P, I, P, I, I, I, P, P, P], I),
         "zq_launch_count": ([], ctypes.c_ulonglong),
         "zq_workspace_reserve": ([ctypes.c_ulonglong], I),
+        "zq_widen_int4_weights": ([P, I, I, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -243,6 +245,17 @@ def gemm_w4a8(Xq, s_tok, Wq4, s_grp, bias=None, Y=None, acc_dbg=None, stream=Non
     """As gemm_w8a8 with packed INT4 weights uint8 [N, K/2]."""
     return _gemm(_lib.zq_gemm_w4a8, "zq_gemm_w4a8", Xq, s_tok, Wq4, s_grp, bias, Wq4.shape[0], Y,
                  acc_dbg, stream, 4)
+
+
+def widen_int4_weights(Wq4, K: int, Wq8=None, stream=None):
+    """Packed INT4 codes uint8 [N, K/2] -> int8 codes [N, K] (zq_widen_int4_weights)."""
+    N = Wq4.shape[0]
+    if Wq8 is None:
+        Wq8 = torch.empty((N, K), dtype=torch.int8, device=Wq4.device)
+    _check(_lib.zq_widen_int4_weights(
+        _dev(Wq4, torch.uint8, (N, K // 2), "Wq4"), N, K, _dev(Wq8, torch.int8, (N, K), "Wq8"),
+        _stream(stream)), "zq_widen_int4_weights")
+    return Wq8
 
 
 def gemm_w8a8_noalloc(Xq, s_tok, Wq, s_grp, bias=None, Y=None, acc_dbg=None, stream=None):

@@ -130,6 +130,20 @@ def test_static_quant_rejects(zq, args, expect):
     assert rc == getattr(zq, "ZQ_ERR_" + expect)
 
 
+@pytest.mark.parametrize("args,expect", [
+    # (Wq4, N, K, Wq8)
+    ((FAKE, 0, 64, FAKE), "SHAPE"),
+    ((FAKE, 16, 48, FAKE), "SHAPE"),
+    ((FAKE, 16, 16, FAKE), "SHAPE"),
+    ((None, 16, 64, FAKE), "NULL"),
+    ((FAKE, 16, 64, None), "NULL"),
+    ((FAKE + 8, 16, 64, FAKE), "ALIGN"),
+])
+def test_widen_int4_rejects(zq, args, expect):
+    rc = zq.lib().zq_widen_int4_weights(*args, None)
+    assert rc == getattr(zq, "ZQ_ERR_" + expect)
+
+
 def test_zero_tokens_is_a_no_op(zq):
     assert zq.lib().zq_bias_act_quant(None, None, 0, 64, 1, None, None, None, None) == zq.ZQ_OK
     assert zq.lib().zq_ln_quant(None, None, None, 0, 64, 1e-5, None, None, None, None) == zq.ZQ_OK

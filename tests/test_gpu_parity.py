@@ -208,6 +208,26 @@ def test_gemm_w4_widened_then_int8(zq, T, N, K, g, pair):
     _check_gemm(zq, T, N, K, g, 4, seed=T + N + pair, path=4, pair=pair)
 
 
+@pytest.mark.parametrize("N,K", [(256, 64), (1000, 4160), (24576, 6144), (3, 32)])
+def test_widen_int4_weights_bit_exact(zq, N, K):
+    """The INT4 unpack step on its own: every widened code equals the oracle's
+    unpacking of the packed bytes, and a W8A8 GEMM on the widened codes equals
+    the W4A8 GEMM on the packed ones."""
+    W = synth.weights(N, K, 0.02, seed=N + K)
+    q, _ = oracle.quantize_weights_groupwise(W.numpy(), max(1, N // 64), 4)
+    packed = torch.from_numpy(oracle.pack_int4(q)).cuda()
+    wide = zq.widen_int4_weights(packed, K)
+    assert_bits_equal(host(wide), oracle.unpack_int4(oracle.pack_int4(q), K))
+    assert_bits_equal(host(wide), q)
+    if N * K <= 1 << 22 and N % 8 == 0:
+        xq, st, _, sg, b = _quant_operands(40, N, K, max(1, N // 64), 4, N)
+        X, S, B = (torch.from_numpy(a).cuda() for a in (xq, st, b))
+        sgd = torch.from_numpy(np.ones(max(1, N // 64), np.float32)).cuda()
+        y8 = zq.gemm_w8a8(X, S, wide, sgd, B)
+        y4 = zq.gemm_w4a8(X, S, packed, sgd, B)
+        assert torch.equal(y8, y4)
+
+
 def test_gemm_w4_widened_after_a_larger_call_and_reserve(zq):
     """The workspace holds the widened codes of the largest call so far; a
     smaller call after it, and calls after an explicit reservation, still
@@ -242,10 +262,11 @@ def test_gemm_cta_pair_tiles(zq, bits, bn, T, N, K):
 @pytest.mark.parametrize("T,N,K,pair", [(2560, 2048, 1024, 2), (2048, 2560, 2048, 1),
                                         (2600, 2056, 1056, 2)])
 def test_gemm_last_wave_split(zq, bits, T, N, K, pair):
-    """A last wave less than half full: its tiles are split along K, their int32
-    partial sums added and dequantized by the finalize kernel (80 pair units
-    over 74 pair slots, 160 single-CTA units over 148 SMs; ragged T, N and K)."""
-    _check_gemm(zq, T, N, K, 8, bits, seed=T + K + pair, pair=pair, bn=256)
+    """A partial last wave whose tiles are split along K (forced here; automatic
+    for long rows), their int32 partial sums added and dequantized by the
+    finalize kernel (80 pair units over 74 pair slots, 160 single-CTA units
+    over 148 SMs; ragged T, N and K)."""
+    _check_gemm(zq, T, N, K, 8, bits, seed=T + K + pair, pair=pair, bn=256, split_k=3)
 
 
 @pytest.mark.parametrize("bits", [8, 4])

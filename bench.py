@@ -384,6 +384,8 @@ class KernelTimer:
         times each in alternation, and the smallest of each is used, so a
         drift of the flush's own time (clocks under the power cap) does not
         land on the kernel."""
+        fn()  # once outside capture: workspaces and launch settings exist first
+        torch.cuda.synchronize()
         g = self._graph(fn)
         tk, tb = [], []
         for _ in range(3):

@@ -655,6 +655,11 @@ def measure_step(zq, weights, T, args, timer, flush_buf, stream, dist_on, inputs
     """Build one layer step at T tokens, record it as a graph, time K steps
     (L2 flushed before each) and every kernel on its own."""
     step = LayerStep(zq, weights, T, torch.device("cuda", torch.cuda.current_device()), inputs)
+    # The per-kernel timings call zq_gemm_w4a8 on its own, which needs more
+    # library workspace than the step (its INT4 widening goes there): size it
+    # for those calls first, so that the step's graph records the final buffer.
+    for it in step.items:
+        step.run_gemm(it)
     graph, graph_error, launches = record_step(step, args.warmup)
     run_step = graph.replay if graph is not None else step.run
     barrier(dist_on)

@@ -152,7 +152,12 @@ zq_status zq_static_quant(const void* X, int T, int K, float amax, int8_t* Xq, f
  * The library workspace is one device buffer per device, grown with
  * cudaMalloc the first time a call needs more than it holds (see
  * zq_workspace_reserve to size it up front); calls that use it on
- * different streams must not overlap.
+ * different streams must not overlap.  Growing it never frees the old
+ * buffer (it stays allocated until the process exits), so a CUDA graph
+ * captured before a growth stays valid.  A call that would grow it while
+ * `stream` is being captured returns ZQ_ERR_UNSUPPORTED and launches
+ * nothing: size the workspace before the capture (an eager call of the
+ * same shape, or zq_workspace_reserve).
  * Requirements: T >= 0 (T == 0 is a no-op), N >= 8, N % 8 == 0,
  * 16 <= K <= 133136, K % 16 == 0 (so that 127*127*K < 2^31), 1 <= g <= N,
  * pointers 16-byte aligned.
@@ -319,7 +324,10 @@ int zq_get_option(int key);
  * plan, plus N * K bytes (rounded up to 256) when zq_gemm_w4a8 widens its
  * codes (T >= 512, or ZQ_OPT_GEMM_PATH = 4); 2 * N * K bytes when an
  * FP16-activation GEMM widens its codes (T >= 1024, or path 4).  Synchronous; call it
- * outside stream capture.  Returns ZQ_ERR_CUDA if the allocation fails.
+ * outside stream capture.  A growth keeps the previous buffer allocated (for
+ * graphs captured with it) and takes at least a quarter more than the
+ * previous size, rounded up to 2 MiB.  Returns ZQ_ERR_CUDA if the
+ * allocation fails.
  */
 zq_status zq_workspace_reserve(unsigned long long bytes);
 

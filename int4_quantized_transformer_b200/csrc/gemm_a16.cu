@@ -758,8 +758,8 @@ zq_status gemm_a16_entry(bool w4, const void* X, const void* Wq, const float* s_
   const void* wsrc = Wq;
   if (pre) {
     void* wide = nullptr;
-    if (library_workspace(static_cast<size_t>(N) * K * 2, &wide) != cudaSuccess)
-      return ZQ_ERR_CUDA;
+    const zq_status wrc = library_workspace(static_cast<size_t>(N) * K * 2, st, &wide);
+    if (wrc != ZQ_OK) return wrc;
     const size_t n16 = static_cast<size_t>(N) * w_inner / 16;
     const int blocks = static_cast<int>(std::min<size_t>((n16 + 255) / 256, 8 * sms));
     const cudaError_t we =

@@ -45,6 +45,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "zq_internal.h"
 #include "zq_ptx.cuh"
@@ -1127,39 +1128,59 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------ host
 
+// The library workspace of one device.  Growing it allocates a new buffer
+// and retires the old one without freeing it: kernels recorded into a CUDA
+// graph before the growth keep their pointers into the old buffer, and the
+// graph stays valid.  Retired buffers are released when the process exits.
+// Each growth takes at least a quarter more than the last size, so the
+// retired buffers together hold less than four times the final size.
 struct Workspace {
   int32_t* ws = nullptr;
   size_t ws_elems = 0;
+  std::vector<void*> retired;
 };
 std::mutex g_ws_mu;
 Workspace g_ws[64];
 
-cudaError_t ensure_workspace(size_t elems, Workspace** out) {
+constexpr size_t kWorkspaceGranule = size_t(1) << 19;  // int32 elements (2 MiB)
+
+// A workspace of at least `elems` int32 elements on the current device.
+// `check_capture`: refuse (ZQ_ERR_UNSUPPORTED) to grow while `st` is being
+// captured into a CUDA graph, since an allocation would end the capture.
+zq_status ensure_workspace(size_t elems, bool check_capture, cudaStream_t st, int32_t** out) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ZQ_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return ZQ_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_ws_mu);
   Workspace& w = g_ws[dev];
   if (w.ws_elems < elems) {
-    if (w.ws) cudaFree(w.ws);
-    w.ws = nullptr;
-    w.ws_elems = 0;
-    e = cudaMalloc(&w.ws, elems * sizeof(int32_t));
-    if (e != cudaSuccess) return e;
-    w.ws_elems = elems;
+    if (check_capture) {
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+        return ZQ_ERR_UNSUPPORTED;
+    }
+    size_t want = std::max(elems, w.ws_elems + w.ws_elems / 4);
+    want = (want + kWorkspaceGranule - 1) / kWorkspaceGranule * kWorkspaceGranule;
+    int32_t* p = nullptr;
+    if (cudaMalloc(&p, want * sizeof(int32_t)) != cudaSuccess) {
+      cudaGetLastError();  // the failed allocation is reported, not left sticky
+      return ZQ_ERR_CUDA;
+    }
+    if (w.ws) w.retired.push_back(w.ws);
+    w.ws = p;
+    w.ws_elems = want;
   }
-  *out = &w;
-  return cudaSuccess;
+  *out = w.ws;
+  return ZQ_OK;
 }
 
 }  // namespace
 
-cudaError_t library_workspace(size_t bytes, void** out) {
-  Workspace* w = nullptr;
-  const cudaError_t e = ensure_workspace((bytes + 3) / 4, &w);
-  if (e == cudaSuccess) *out = w->ws;
-  return e;
+zq_status library_workspace(size_t bytes, cudaStream_t st, void** out) {
+  int32_t* p = nullptr;
+  const zq_status rc = ensure_workspace((bytes + 3) / 4, true, st, &p);
+  if (rc == ZQ_OK) *out = p;
+  return rc;
 }
 
 namespace {
@@ -1610,9 +1631,8 @@ zq_status gemm_entry(bool w4, const int8_t* Xq, const float* s_tok, const void* 
   const size_t wide_ints = ch.widen ? (static_cast<size_t>(N) * K + 255) / 256 * 64 : 0;
   int32_t* ws = nullptr;
   if (partials > 0 || wide_ints > 0) {
-    Workspace* w = nullptr;
-    if (ensure_workspace(wide_ints + partials, &w) != cudaSuccess) return ZQ_ERR_CUDA;
-    ws = w->ws;
+    rc = ensure_workspace(wide_ints + partials, true, st, &ws);
+    if (rc != ZQ_OK) return rc;
   }
   if (ch.widen) {
     const size_t n16 = static_cast<size_t>(N) * (K / 2) / 16;
@@ -1647,9 +1667,9 @@ extern "C" zq_status zq_widen_int4_weights(const uint8_t* Wq4, int N, int K, int
 }
 
 extern "C" zq_status zq_workspace_reserve(unsigned long long bytes) {
-  zq::Workspace* w = nullptr;
+  int32_t* p = nullptr;
   if (bytes == 0) return ZQ_OK;
-  return zq::ensure_workspace((bytes + 3) / 4, &w) == cudaSuccess ? ZQ_OK : ZQ_ERR_CUDA;
+  return zq::ensure_workspace((bytes + 3) / 4, false, nullptr, &p);
 }
 
 extern "C" zq_status zq_gemm_w8a8(const int8_t* Xq, const float* s_tok, const int8_t* Wq,

@@ -596,11 +596,6 @@ cudaError_t launch_ln_w(int vpt, const __half* X, const __half* g, const __half*
   }
 }
 
-// LayerNorm rows of 32 * W vectors with W in {3, 6, 12, 24} get W warps per
-// row pair and one vector per thread (kLnOneVectorPerThread), else the
-// power-of-two rule below.
-constexpr bool kLnOneVectorPerThread = false;
-
 // Warps per row so that each thread keeps at most 4 vectors of 8 halves
 // (3 for the two-row LayerNorm kernel, which holds both rows); act < 0
 // selects the LayerNorm (gamma non-NULL) or quant-only form; sa >= 0 is a
@@ -613,23 +608,6 @@ cudaError_t launch_row_quant(const __half* xg, const __half* gg, const __half* b
   int W = 1;
   while (W < 32 && 32 * W * vmax < nvec) W *= 2;
   const int vpt = (nvec + 32 * W - 1) / (32 * W);
-  if (gg && kLnOneVectorPerThread && nvec % 32 == 0) {
-    switch (nvec / 32) {
-      case 3: return launch_ln_rows2<3, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
-      case 6: return launch_ln_rows2<6, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
-      case 12: return launch_ln_rows2<12, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
-      case 24: return launch_ln_rows2<24, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
-      case 1: case 2: case 4: case 8: case 16: case 32:
-        W = nvec / 32;
-        return W == 1 ? launch_ln_rows2<1, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st)
-             : W == 2 ? launch_ln_rows2<2, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st)
-             : W == 4 ? launch_ln_rows2<4, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st)
-             : W == 8 ? launch_ln_rows2<8, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st)
-             : W == 16 ? launch_ln_rows2<16, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st)
-                       : launch_ln_rows2<32, 1>(xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);
-      default: break;
-    }
-  }
   if (gg) {
     switch (W) {
       case 1: return launch_ln_w<1>(vpt, xg, gg, bg, T, K, eps, Xq, s_tok, yg, st);

@@ -147,7 +147,7 @@ const char* zq_status_str(int s) {
   }
 }
 
-int zq_abi_version(void) { return 104; }
+int zq_abi_version(void) { return 105; }
 
 zq_status zq_set_option(int key, int value) {
   if (key < ZQ_OPT_GEMM_PATH || key > ZQ_OPT_CTA_PAIR) return ZQ_ERR_UNSUPPORTED;

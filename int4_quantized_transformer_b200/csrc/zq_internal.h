@@ -34,10 +34,11 @@ cudaError_t launch_gemv_a16(int bits, const void* X, const void* W, const float*
                             int max_ctas, cudaStream_t st);
 int option(int key);
 // The library workspace of the current device (gemm_i8.cu): at least
-// `bytes` bytes, grown with cudaMalloc when a call needs more than it holds.
+// `bytes` bytes, grown with cudaMalloc when a call needs more than it holds
+// (ZQ_ERR_UNSUPPORTED instead while `st` is being captured into a graph).
 // One buffer per device; calls that use it on different streams must not
 // overlap.
-cudaError_t library_workspace(size_t bytes, void** out);
+zq_status library_workspace(size_t bytes, cudaStream_t st, void** out);
 // Counts one kernel launch issued by the library (zq_launch_count).
 void count_launch();
 

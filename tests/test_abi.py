@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(zq):
 
 
 def test_status_strings_and_version(zq):
-    assert zq.abi_version() == 104
+    assert zq.abi_version() == 105
     for s in range(7):
         assert zq.status_str(s).startswith("ZQ_")
     assert "unknown" in zq.status_str(99)

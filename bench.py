@@ -63,11 +63,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture of a GEMM with a cold L2, keyed by (layer, gemm, T); valid
-# only for the GEMM source it was taken with (sha256 prefix of the .cu file
-# named in "file").
-NCU_TRAFFIC: dict = {}
+# DRAM bytes per GEMM call (dram__bytes_read.sum + dram__bytes_write.sum,
+# summed over the call's kernels) from one ncu capture with a cold L2, keyed
+# by (layer, gemm, T); valid only for the GEMM source it was taken with
+# (sha256 prefix of the .cu file named in "file").
+NCU_TRAFFIC: dict = {
+    # zq_gemm_w4a8, GPT-NeoX FFN2 24576->6144 at T=4096: widen_w4_kernel
+    # (76957952 read + 92952320 written), gemm_i8_kernel (744837888 +
+    # 44560896), tail_finalize_kernel (18382592 + 0)
+    ("neox20b", "ffn2", 4096): {"file": "gemm_i8.cu", "source": "317b3260ed0e",
+                                "bytes": 977691648},
+}
 
 
 def _source_hash(name: str) -> str:
@@ -204,12 +210,21 @@ class LayerWeights:
     def __init__(self, zq, layer, device, keep_fp16=True):
         self.layer = layer
         self.items = []
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
+        # device time of the weight quantization alone (the synthetic fp16
+        # weights are drawn on the host and copied in outside the events)
+        self.wquant_ms = 0.0
+        z = torch.zeros((8, 64), dtype=torch.float16, device=device)
+        for bits in (8, 4):  # the first launch of each kernel loads it: keep that out of the events
+            zq.quantize_weights_groupwise(z, 1, bits)
         for i, s in enumerate(synth.LAYERS[layer].gemms):
             gi = synth.gemm_inputs(layer, i, 1)
             W = gi.W.to(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
             Wq, sg = zq.quantize_weights_groupwise(W, s.g, s.bits)
+            e1.record()
+            e1.synchronize()
+            self.wquant_ms += e0.elapsed_time(e1)
             self.items.append({
                 "spec": s, "W16": W if keep_fp16 else None, "Wq": Wq, "s_grp": sg,
                 "b": gi.b.to(device),
@@ -217,8 +232,6 @@ class LayerWeights:
                 "beta": None if gi.beta is None else gi.beta.to(device),
             })
             del W
-        torch.cuda.synchronize()
-        self.wquant_s = time.perf_counter() - t0
 
 
 class LayerStep:
@@ -732,7 +745,7 @@ def gpu_arm(args, dist_on, rank, world):
     if "gemm_us" in fp16:
         fp16["gemm_speedup"] = round(sum(fp16["gemm_us"].values()) / (gemm_ms * 1e3), 3)
         fp16["step_speedup"] = round(fp16["step_us"] / (ms_per_step * 1e3), 3)
-    wquant_ms = weights.wquant_s * 1e3
+    wquant_ms = weights.wquant_ms
     summary = step_summary(step, kern, per_step, launches)
     del graph, step
 

@@ -1263,8 +1263,23 @@ Plan plan_wrows(int T, int N, int K, int sms, int forced_split, bool w4) {
     const int s_eff = ceil_div(k_stages, sps);
     const int units = tiles * s_eff;
     const int waves = ceil_div(units, sms);
-    // the unit time is set by streaming its weights (HBM-bound): count bytes
-    const double cost = waves * (sps * kps + 2.0) + (s_eff > 1 ? 1.0 : 0.0);
+    double cost;
+    if (w4) {
+      // the unit time is set by its widening pipeline: count stages
+      cost = waves * (sps * kps + 2.0) + (s_eff > 1 ? 1.0 : 0.0);
+    } else {
+      // INT8 weights, in microseconds (fitted to B200 kernel timings after an
+      // L2 flush, T = 8 to 64): the weights stream at the lower of 5.5 TB/s
+      // over the GPU and 55 GB/s into one CTA (the operand bytes of its
+      // stages); a K split costs 3 us + 0.1 us per token column of the tile
+      // (the partial sums' stores and the finalize kernel), and each further
+      // unit a persistent CTA takes on about 0.9 us
+      const double w_stage = static_cast<double>(BM) * BK;
+      const double cta_bytes = waves * sps * (w_stage + static_cast<double>(bn) * BK);
+      const double all_bytes = static_cast<double>(tiles) * k_stages * w_stage;
+      cost = std::max(all_bytes / 5.5e6, cta_bytes / 5.5e4) +
+             (s_eff > 1 ? 3.0 + 0.1 * bn : 0.0) + 0.9 * (waves - 1);
+    }
     if (cost < best - 1e-9) {
       best = cost;
       best_s = s_eff;

@@ -182,6 +182,18 @@ __device__ __forceinline__ float habs_max(uint32_t m2) {
   return fmaxf(fabsf(f.x), fabsf(f.y));
 }
 
+// L2 prefetch of one fp16 row of K values (K % 8 == 0, 16-byte aligned),
+// in bulk requests of at most 64 KB.
+__device__ __forceinline__ void prefetch_row_l2(const __half* v, int K) {
+  const char* p = reinterpret_cast<const char*>(v);
+  for (uint32_t left = static_cast<uint32_t>(K) * 2u; left > 0;) {
+    const uint32_t n = left < 65536u ? left : 65536u;
+    bulk_prefetch_l2(p, n);
+    p += n;
+    left -= n;
+  }
+}
+
 // ------------------------------------------------- token quantization only
 
 // One row per group of W warps, VPT 16-byte vectors (8 halves) per thread:
@@ -205,6 +217,8 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32, (W >= 8 ? 2048 / (W * 3
   const int warp_in_row = j / 32;
   const int lane = threadIdx.x & 31;
   const int nvec = K / 8;
+  // the bias of the bias-add / GeLU form, as gamma and beta in ln_rows2_kernel
+  if (act_bias && blockIdx.x == 0 && threadIdx.x == 0) prefetch_row_l2(act_bias, K);
   grid_dependency_wait();
   grid_launch_dependents();
 
@@ -378,6 +392,14 @@ __global__ void __launch_bounds__((W >= 8 ? W : 8) * 32)
   const int warp_in_row = j / 32;
   const int lane = threadIdx.x & 31;
   const int nvec = K / 8;
+  // gamma and beta are read only after the row statistics: ask L2 for them
+  // now, before waiting for the previous kernel of the stream, so that their
+  // DRAM latency overlaps the wait and the reductions (an L2 prefetch, which
+  // every kernel's writes reach coherently, so a stale read is impossible).
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    prefetch_row_l2(gamma, K);
+    if (beta) prefetch_row_l2(beta, K);
+  }
   grid_dependency_wait();
   grid_launch_dependents();
 

